@@ -1,0 +1,704 @@
+// C ABI of libdg: argument checks, device memory, weight initialisation and
+// the orchestration of one canvas denoising pass on a single stream.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "dg.h"
+#include "dg_kernels.h"
+
+using namespace dg;
+
+namespace {
+
+constexpr int kGroupedTile = 128;   // B rows per grouped-GEMM tile
+constexpr int kMaxAttnChunks = 16;
+constexpr int kMaxSplits = 16;
+
+std::string g_create_error;
+
+struct Layer {
+  bf16 *wqkv = nullptr, *wo = nullptr, *wr = nullptr, *wgu = nullptr, *wd = nullptr;
+  float *ln_in = nullptr, *ln_post = nullptr, *ln_ff = nullptr;
+  CUtensorMap m_qkv, m_o, m_r, m_gu, m_d;
+  const bf16* kp = nullptr;
+  const bf16* vp = nullptr;
+  int kv_batch = 0, kv_P = 0;
+};
+
+}  // namespace
+
+struct dg_ctx {
+  dg_config cfg;
+  cudaStream_t stream = nullptr;
+  int device = 0, num_sms = 148;
+  std::string err;
+  size_t bytes = 0;
+  std::vector<void*> allocs;
+  bool weights_ready = false;
+
+  int Tmax = 0, NQKV = 0, G = 0;
+  bf16* embed = nullptr;
+  float* ln_final = nullptr;
+  std::vector<Layer> layers;
+  CUtensorMap m_embed;
+
+  // workspace
+  float* h = nullptr;
+  bf16* x = nullptr;
+  float* part = nullptr;
+  size_t part_elems = 0;
+  bf16 *q = nullptr, *kc = nullptr, *vc = nullptr;
+  float *attn_po = nullptr, *attn_ml = nullptr;
+  bf16* attn_o = nullptr;
+  bf16* xperm = nullptr;
+  float* router_logits = nullptr;
+  int32_t* idx = nullptr;
+  float* w = nullptr;
+  uint32_t* bitmap = nullptr;
+  int32_t *offsets_r = nullptr, *offsets_g = nullptr, *chunk_prefix = nullptr;
+  int32_t *perm = nullptr, *inv = nullptr;
+  bf16* H = nullptr;
+  float* Y = nullptr;
+  float *head_m = nullptr, *head_s = nullptr;
+  int* head_a = nullptr;
+  float* conf = nullptr;
+  int32_t* tok = nullptr;
+  int32_t* canvas_dev = nullptr;
+  uint8_t* committed_dev = nullptr;
+  int* err_dev = nullptr;
+  float *rope_cos = nullptr, *rope_sin = nullptr;
+  int rope_P = -1;
+  float* router_bias = nullptr;
+  bool has_bias = false;
+  CUtensorMap m_x_b, m_x_a, m_attn_o_b, m_xperm_b, m_H_b;
+
+  int last_T = 0, last_B = 0, launches = 0;
+};
+
+namespace {
+
+int fail(dg_ctx* c, int code, const std::string& msg) {
+  if (c) c->err = msg;
+  else g_create_error = msg;
+  return code;
+}
+
+#define DG_CUDA(ctx, call)                                                             \
+  do {                                                                                 \
+    cudaError_t e_ = (call);                                                           \
+    if (e_ != cudaSuccess)                                                             \
+      return fail(ctx, DG_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+
+#define DG_LAUNCH(ctx, call)   \
+  do {                         \
+    ++(ctx)->launches;         \
+    DG_CUDA(ctx, call);        \
+  } while (0)
+
+bool ctx_alloc(dg_ctx* c, void** p, size_t bytes) {
+  *p = nullptr;
+  if (bytes == 0) bytes = 16;
+  bytes = (bytes + 255) & ~size_t(255);
+  if (c->cfg.alloc_limit_bytes && c->bytes + bytes > c->cfg.alloc_limit_bytes) return false;
+  if (cudaMalloc(p, bytes) != cudaSuccess) {
+    *p = nullptr;
+    cudaGetLastError();
+    return false;
+  }
+  c->allocs.push_back(*p);
+  c->bytes += bytes;
+  return true;
+}
+
+template <class T>
+bool alloc_n(dg_ctx* c, T** p, size_t n) {
+  return ctx_alloc(c, reinterpret_cast<void**>(p), n * sizeof(T));
+}
+
+void free_all(dg_ctx* c) {
+  for (void* p : c->allocs) cudaFree(p);
+  c->allocs.clear();
+}
+
+bool is_global(const dg_config& c, int l) { return (l + 1) % c.global_every == 0; }
+
+int n_rot_pairs(const dg_config& c, int l) {
+  if (!c.rope_enabled) return 0;
+  const int half = c.head_dim / 2;
+  if (is_global(c, l)) return (int)std::ceil((double)c.prope_fraction * half);
+  return half;
+}
+
+std::string check_config(const dg_config& c) {
+  if (c.n_layers < 1) return "n_layers must be >= 1";
+  if (c.d_model < 128 || c.d_model % 64 || c.d_model > 4096) return "d_model must be a multiple of 64 in [128, 4096]";
+  if (c.d_ff < 64 || c.d_ff % 64) return "d_ff must be a positive multiple of 64";
+  if (c.head_dim != 64 && c.head_dim != 128 && c.head_dim != 256) return "head_dim must be 64, 128 or 256";
+  if (c.n_kv_heads < 1 || c.n_q_heads < 1 || c.n_q_heads % c.n_kv_heads) return "n_q_heads must be a positive multiple of n_kv_heads";
+  if (c.n_experts < 1 || c.n_experts > 256) return "n_experts must be in [1, 256]";
+  if (c.top_k < 1 || c.top_k > c.n_experts || c.top_k > 32) return "top_k must be in [1, min(n_experts, 32)]";
+  if (c.n_shared != 0 && c.n_shared != 1) return "n_shared must be 0 or 1";
+  if (c.vocab < 2) return "vocab must be >= 2";
+  if (c.canvas_len < 1 || c.canvas_len > 256) return "canvas_len must be in [1, 256]";
+  if (c.max_batch < 1 || (long long)c.max_batch * c.canvas_len > 4096) return "max_batch * canvas_len must be in [1, 4096]";
+  if (c.max_prompt < 1) return "max_prompt must be >= 1";
+  if (c.mask_id < 0 || c.mask_id >= c.vocab) return "mask_id must be in [0, vocab)";
+  if (c.window < 1 || c.global_every < 1) return "window and global_every must be >= 1";
+  if (!(c.rms_eps >= 0.f) || !(c.rope_theta > 0.f)) return "rms_eps must be >= 0 and rope_theta > 0";
+  if (!(c.prope_fraction >= 0.f && c.prope_fraction <= 1.f)) return "prope_fraction must be in [0, 1]";
+  if (!(c.weight_std > 0.0)) return "weight_std must be > 0";
+  return "";
+}
+
+int choose_splits(int base_tiles, int n_kb, int num_sms) {
+  int best = 1;
+  double best_cost = 1e30;
+  for (int ks = 1; ks <= kMaxSplits && ks <= n_kb; ++ks) {
+    const int tiles = base_tiles * ks;
+    const int waves = (tiles + num_sms - 1) / num_sms;
+    const double cost = (double)waves / ks * (1.0 + 0.02 * ks);  // small penalty for partial traffic
+    if (cost < best_cost - 1e-9) { best_cost = cost; best = ks; }
+  }
+  return best;
+}
+
+// Dense swap-AB projection: part[s][n][m] = X[n] . W[m] over split s.
+int run_dense(dg_ctx* c, const CUtensorMap& mA, const CUtensorMap& mB, int M, int N, int K,
+              int* splits_out) {
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.mode = GEMM_DENSE;
+  a.M = M; a.N = N; a.K = K; a.n_kb = K / 64;
+  a.n_tile = std::min(256, (N + 31) / 32 * 32);
+  a.m_slabs = (M + 127) / 128;
+  const int n_chunks = (N + a.n_tile - 1) / a.n_tile;
+  a.k_splits = choose_splits(a.m_slabs * n_chunks, a.n_kb, c->num_sms);
+  if ((size_t)a.k_splits * N * M > c->part_elems) a.k_splits = 1;
+  a.out_f32 = c->part;
+  a.err = c->err_dev;
+  gemm_plan_smem(a);
+  const int tiles = a.m_slabs * n_chunks * a.k_splits;
+  DG_LAUNCH(c, gemm_tc_launch(mA, mB, a, std::min(tiles, c->num_sms), c->stream));
+  *splits_out = a.k_splits;
+  return DG_OK;
+}
+
+int run_grouped(dg_ctx* c, int mode, const CUtensorMap& mA, const CUtensorMap& mB, int K, int M,
+                int T) {
+  const dg_config& cf = c->cfg;
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.mode = mode;
+  a.K = K; a.n_kb = K / 64;
+  a.M = M;
+  a.n_tile = kGroupedTile;
+  a.m_slabs = (M + 127) / 128;
+  a.n_groups = cf.n_experts + 1;
+  a.offsets = c->offsets_g;
+  a.chunk_prefix = c->chunk_prefix;
+  a.F = cf.d_ff;
+  a.out_f32 = c->Y;
+  a.out_bf16 = c->H;
+  a.err = c->err_dev;
+  (void)T;
+  gemm_plan_smem(a);
+  DG_LAUNCH(c, gemm_tc_launch(mA, mB, a, c->num_sms, c->stream));
+  return DG_OK;
+}
+
+// One decoder block on c->h / c->x (x = input-normed h).  On return h is the
+// block output and x = bf16(rmsnorm(h) * w_next) (or bf16(h) when w_next is NULL).
+int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
+  const dg_config& cf = c->cfg;
+  Layer& L = c->layers[l];
+  const int Tc = cf.canvas_len, T = B * Tc, d = cf.d_model, dh = cf.head_dim;
+  const int Hq = cf.n_q_heads, Hkv = cf.n_kv_heads, E = cf.n_experts, k = cf.top_k;
+  const int P = L.kv_P;
+  int splits = 1, rc;
+
+  // q/k/v projections, RoPE / p-RoPE on the canvas rows
+  if ((rc = run_dense(c, L.m_qkv, c->m_x_b, c->NQKV, T, d, &splits)) != DG_OK) return rc;
+  DG_LAUNCH(c, launch_qkv_rope(c->part, splits, T, Tc, Hq, Hkv, dh, n_rot_pairs(cf, l), c->rope_cos,
+                               c->rope_sin, c->q, c->kc, c->vc, c->stream));
+
+  // one softmax over the visible prompt keys and all canvas keys, split-KV
+  AttnArgs at;
+  memset(&at, 0, sizeof(at));
+  at.q = c->q; at.kc = c->kc; at.vc = c->vc; at.kp = L.kp; at.vp = L.vp;
+  at.B = B; at.Hq = Hq; at.Hkv = Hkv; at.Tc = Tc; at.P = P; at.dh = dh;
+  at.n_vis = is_global(cf, l) ? P : std::min(cf.window, P);
+  const int NK = at.n_vis + Tc;
+  const int q_tiles = (Hq / Hkv * Tc + 63) / 64;
+  const int base = q_tiles * B * Hkv;
+  int nch = std::max(1, std::min(kMaxAttnChunks, (2 * c->num_sms + base - 1) / base));
+  nch = std::min(nch, (NK + 63) / 64);
+  at.chunk_keys = ((NK + nch - 1) / nch + 63) / 64 * 64;
+  at.n_chunks = (NK + at.chunk_keys - 1) / at.chunk_keys;
+  at.part_o = c->attn_po; at.part_ml = c->attn_ml;
+  at.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)dh));
+  DG_LAUNCH(c, launch_attention(at, c->stream));
+  DG_LAUNCH(c, launch_attn_merge(at, c->attn_o, c->stream));
+
+  // output projection, post-attention norm + residual, pre-FFN norm
+  if ((rc = run_dense(c, L.m_o, c->m_attn_o_b, d, T, Hq * dh, &splits)) != DG_OK) return rc;
+  DG_LAUNCH(c, launch_post_attn(c->part, splits, T, d, L.ln_post, L.ln_ff, cf.rms_eps, c->h,
+                                c->xperm, c->stream));
+
+  // router
+  if ((rc = run_dense(c, L.m_r, c->m_xperm_b, E, T, d, &splits)) != DG_OK) return rc;
+  DG_LAUNCH(c, launch_router_topk(c->part, splits, c->has_bias ? c->router_bias : nullptr, T, E,
+                                  k, c->router_logits, c->idx, c->w, c->bitmap, c->stream));
+  DG_LAUNCH(c, launch_router_sort(c->idx, c->bitmap, T, E, k, cf.n_shared, kGroupedTile,
+                                  c->offsets_r, c->offsets_g, c->chunk_prefix, c->perm, c->inv,
+                                  c->err_dev, c->stream));
+  DG_LAUNCH(c, launch_moe_gather(c->xperm, c->perm, T, k, d, c->stream));
+
+  // experts (group 0 = shared expert on all rows), SiLU-gated, then down + combine
+  if ((rc = run_grouped(c, GEMM_GATEUP, L.m_gu, c->m_xperm_b, d, 2 * cf.d_ff, T)) != DG_OK) return rc;
+  if ((rc = run_grouped(c, GEMM_DOWN, L.m_d, c->m_H_b, cf.d_ff, d, T)) != DG_OK) return rc;
+  DG_LAUNCH(c, launch_moe_combine(c->Y, c->w, c->inv, T, k, cf.n_shared, d, c->h, w_next,
+                                  cf.rms_eps, c->x, c->stream));
+  return DG_OK;
+}
+
+int check_prompt_state(dg_ctx* c, int batch) {
+  const dg_config& cf = c->cfg;
+  int P = -1;
+  for (int l = 0; l < cf.n_layers; ++l) {
+    const Layer& L = c->layers[l];
+    if (!L.kp) return fail(c, DG_ERR_BAD_STATE, "prompt KV not set for layer " + std::to_string(l));
+    if (L.kv_batch != batch)
+      return fail(c, DG_ERR_BAD_STATE, "batch differs from the batch of the prompt KV");
+    if (P >= 0 && L.kv_P != P)
+      return fail(c, DG_ERR_BAD_STATE, "all layers need the same prompt length");
+    P = L.kv_P;
+  }
+  return DG_OK;
+}
+
+int ensure_rope(dg_ctx* c, int P) {
+  if (c->rope_P != P) {
+    DG_LAUNCH(c, launch_rope_table(c->rope_cos, c->rope_sin, c->cfg.canvas_len,
+                                   c->cfg.head_dim / 2, P, (double)c->cfg.rope_theta, c->stream));
+    c->rope_P = P;
+  }
+  return DG_OK;
+}
+
+// Full pass on c->canvas_dev (batch B), conf/tok into c->conf / c->tok, commit in place.
+int run_step(dg_ctx* c, int B, int steps_left) {
+  const dg_config& cf = c->cfg;
+  const int T = B * cf.canvas_len, d = cf.d_model;
+  int rc;
+  c->launches = 0;
+  if ((rc = ensure_rope(c, c->layers[0].kv_P)) != DG_OK) return rc;
+  DG_LAUNCH(c, launch_embed_norm(c->canvas_dev, c->embed, nullptr, cf.vocab, T, d,
+                                 c->layers[0].ln_in, cf.rms_eps, c->h, c->x, c->err_dev,
+                                 c->stream));
+  for (int l = 0; l < cf.n_layers; ++l) {
+    const float* w_next = (l + 1 < cf.n_layers) ? c->layers[l + 1].ln_in : c->ln_final;
+    if ((rc = run_layer(c, l, B, w_next)) != DG_OK) return rc;
+  }
+  // tied vocab head with the fused (max, argmax, sum-exp) reduction
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.mode = GEMM_HEAD;
+  a.K = d; a.n_kb = d / 64;
+  a.T = T; a.vocab = cf.vocab; a.mask_id = cf.mask_id;
+  a.n_vblocks = (cf.vocab + 255) / 256;
+  a.n_tblocks = (T + 255) / 256;
+  a.head_m = c->head_m; a.head_s = c->head_s; a.head_a = c->head_a;
+  a.err = c->err_dev;
+  gemm_plan_smem(a);
+  const int tiles = a.n_vblocks * a.n_tblocks;
+  DG_LAUNCH(c, gemm_tc_launch(c->m_x_a, c->m_embed, a, std::min(tiles, c->num_sms), c->stream));
+  DG_LAUNCH(c, launch_head_merge(c->head_m, c->head_s, c->head_a, a.n_vblocks, T, c->conf,
+                                 c->tok, c->stream));
+  DG_LAUNCH(c, launch_commit(c->conf, c->tok, c->canvas_dev, c->committed_dev, B, cf.canvas_len,
+                             steps_left, nullptr, cf.mask_id, c->stream));
+  c->last_T = T;
+  c->last_B = B;
+  return DG_OK;
+}
+
+int read_device_error(dg_ctx* c) {
+  int h = 0;
+  DG_CUDA(c, cudaMemcpyAsync(&h, c->err_dev, sizeof(int), cudaMemcpyDeviceToHost, c->stream));
+  DG_CUDA(c, cudaStreamSynchronize(c->stream));
+  if (h != 0) {
+    DG_CUDA(c, cudaMemsetAsync(c->err_dev, 0, sizeof(int), c->stream));
+    DG_CUDA(c, cudaStreamSynchronize(c->stream));
+    if (h == kErrTimeout) return fail(c, DG_ERR_TIMEOUT, "a bounded device wait gave up");
+    return fail(c, DG_ERR_DEVICE_FAULT, "a kernel flagged an out-of-range index");
+  }
+  return DG_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
+  if (!cfg || !out) return fail(nullptr, DG_ERR_INVALID_ARG, "null argument");
+  const std::string why = check_config(*cfg);
+  if (!why.empty()) return fail(nullptr, DG_ERR_INVALID_ARG, why);
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+    cudaGetLastError();
+    return fail(nullptr, DG_ERR_CUDA, "no CUDA device");
+  }
+  dg_ctx* c = new (std::nothrow) dg_ctx();
+  if (!c) return fail(nullptr, DG_ERR_OOM, "host allocation failed");
+  c->cfg = *cfg;
+  c->stream = static_cast<cudaStream_t>(cuda_stream);
+  cudaGetDevice(&c->device);
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, c->device) != cudaSuccess) {
+    delete c;
+    return fail(nullptr, DG_ERR_CUDA, "cudaGetDeviceProperties failed");
+  }
+  if (prop.major != 10) {
+    delete c;
+    return fail(nullptr, DG_ERR_UNSUPPORTED, "needs an sm_100 (B200) device");
+  }
+  c->num_sms = prop.multiProcessorCount;
+  const dg_config& cf = c->cfg;
+  const int d = cf.d_model, F = cf.d_ff, dh = cf.head_dim, E = cf.n_experts, k = cf.top_k;
+  const int Hq = cf.n_q_heads, Hkv = cf.n_kv_heads;
+  c->Tmax = cf.max_batch * cf.canvas_len;
+  c->NQKV = (Hq + 2 * Hkv) * dh;
+  c->G = E + 1;
+  const size_t T = c->Tmax, V = cf.vocab;
+  // Row counts of TMA-read buffers are padded so that no box is taller than its tensor.
+  const size_t Tp = std::max<size_t>(128, (T + 127) / 128 * 128);
+  const size_t Er = (size_t)std::max(E, 128);
+  bool ok = true;
+  ok &= alloc_n(c, &c->embed, V * d);
+  ok &= alloc_n(c, &c->ln_final, d);
+  c->layers.resize(cf.n_layers);
+  for (auto& L : c->layers) {
+    ok &= alloc_n(c, &L.wqkv, (size_t)c->NQKV * d);
+    ok &= alloc_n(c, &L.wo, (size_t)d * Hq * dh);
+    ok &= alloc_n(c, &L.wr, Er * d);
+    ok &= alloc_n(c, &L.wgu, (size_t)c->G * 2 * F * d);
+    ok &= alloc_n(c, &L.wd, (size_t)c->G * d * F);
+    ok &= alloc_n(c, &L.ln_in, d);
+    ok &= alloc_n(c, &L.ln_post, d);
+    ok &= alloc_n(c, &L.ln_ff, d);
+    if (!ok) break;
+  }
+  const size_t rows_moe = std::max<size_t>(128, (size_t)(k + 1) * T);
+  c->part_elems = std::max({(size_t)kMaxSplits * T * c->NQKV, (size_t)kMaxSplits * T * d,
+                            (size_t)kMaxSplits * T * E});
+  if (ok) {
+    ok &= alloc_n(c, &c->h, T * d);
+    ok &= alloc_n(c, &c->x, Tp * d);
+    ok &= alloc_n(c, &c->part, c->part_elems);
+    ok &= alloc_n(c, &c->q, T * Hq * dh);
+    ok &= alloc_n(c, &c->kc, T * Hkv * dh);
+    ok &= alloc_n(c, &c->vc, T * Hkv * dh);
+    ok &= alloc_n(c, &c->attn_po, (size_t)kMaxAttnChunks * T * Hq * dh);
+    ok &= alloc_n(c, &c->attn_ml, (size_t)kMaxAttnChunks * T * Hq * 2);
+    ok &= alloc_n(c, &c->attn_o, Tp * Hq * dh);
+    ok &= alloc_n(c, &c->xperm, rows_moe * d);
+    ok &= alloc_n(c, &c->router_logits, T * E);
+    ok &= alloc_n(c, &c->idx, T * k);
+    ok &= alloc_n(c, &c->w, T * k);
+    ok &= alloc_n(c, &c->bitmap, (size_t)E * ((T + 31) / 32));
+    ok &= alloc_n(c, &c->offsets_r, E + 1);
+    ok &= alloc_n(c, &c->offsets_g, E + 2);
+    ok &= alloc_n(c, &c->chunk_prefix, E + 2);
+    ok &= alloc_n(c, &c->perm, T * k);
+    ok &= alloc_n(c, &c->inv, T * k);
+    ok &= alloc_n(c, &c->H, rows_moe * F);
+    ok &= alloc_n(c, &c->Y, rows_moe * d);
+    const size_t nvb = (V + 255) / 256;
+    ok &= alloc_n(c, &c->head_m, nvb * T);
+    ok &= alloc_n(c, &c->head_s, nvb * T);
+    ok &= alloc_n(c, &c->head_a, nvb * T);
+    ok &= alloc_n(c, &c->conf, T);
+    ok &= alloc_n(c, &c->tok, T);
+    ok &= alloc_n(c, &c->canvas_dev, T);
+    ok &= alloc_n(c, &c->committed_dev, T);
+    ok &= alloc_n(c, &c->err_dev, 4);
+    ok &= alloc_n(c, &c->rope_cos, (size_t)cf.canvas_len * dh / 2);
+    ok &= alloc_n(c, &c->rope_sin, (size_t)cf.canvas_len * dh / 2);
+    ok &= alloc_n(c, &c->router_bias, E);
+  }
+  if (!ok) {
+    const size_t have = c->bytes;
+    free_all(c);
+    delete c;
+    return fail(nullptr, DG_ERR_OOM,
+                "device allocation failed or passed alloc_limit_bytes (after " +
+                    std::to_string(have) + " bytes)");
+  }
+  // zero the scratch that kernels accumulate into or read before writing
+  cudaMemset(c->bitmap, 0, (size_t)E * ((T + 31) / 32) * 4);
+  cudaMemset(c->err_dev, 0, 16);
+  cudaMemset(c->xperm, 0, rows_moe * d * 2);
+  cudaMemset(c->H, 0, rows_moe * F * 2);
+  cudaMemset(c->x, 0, Tp * d * 2);
+  cudaMemset(c->attn_o, 0, Tp * Hq * dh * 2);
+  for (auto& L : c->layers) cudaMemset(L.wr, 0, Er * d * 2);
+  // tensor maps (weights: A operands, 128-row boxes; activations: B operands, 32-row boxes)
+  ok = make_tmap_2d(&c->m_embed, c->embed, d, V, 256);
+  for (auto& L : c->layers) {
+    ok &= make_tmap_2d(&L.m_qkv, L.wqkv, d, c->NQKV, 128);
+    ok &= make_tmap_2d(&L.m_o, L.wo, (uint64_t)Hq * dh, d, 128);
+    ok &= make_tmap_2d(&L.m_r, L.wr, d, Er, 128);
+    ok &= make_tmap_3d(&L.m_gu, L.wgu, d, 2 * F, c->G, 128);
+    ok &= make_tmap_3d(&L.m_d, L.wd, F, d, c->G, 128);
+  }
+  ok &= make_tmap_2d(&c->m_x_b, c->x, d, Tp, 32);
+  ok &= make_tmap_2d(&c->m_x_a, c->x, d, Tp, 128);
+  ok &= make_tmap_2d(&c->m_attn_o_b, c->attn_o, (uint64_t)Hq * dh, Tp, 32);
+  ok &= make_tmap_2d(&c->m_xperm_b, c->xperm, d, rows_moe, 32);
+  ok &= make_tmap_2d(&c->m_H_b, c->H, F, rows_moe, 32);
+  if (cudaDeviceSynchronize() != cudaSuccess || !ok) {
+    cudaGetLastError();
+    free_all(c);
+    delete c;
+    return fail(nullptr, DG_ERR_CUDA, "tensor map creation or initial memset failed");
+  }
+  *out = c;
+  return DG_OK;
+}
+
+int dg_init_weights(dg_ctx* c, uint64_t seed) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  const dg_config& cf = c->cfg;
+  const int d = cf.d_model, F = cf.d_ff, dh = cf.head_dim, E = cf.n_experts;
+  const int Hq = cf.n_q_heads, Hkv = cf.n_kv_heads;
+  const float scale = (float)(cf.weight_std * std::sqrt(3.0) / 65536.0);
+  auto key = [&](unsigned long long tid) { return stream_key_host(seed, tid); };
+  auto ltid = [](int l, int kind) { return 64ull * (unsigned long long)(l + 1) + (unsigned)kind; };
+  InitArgs a;
+  memset(&a, 0, sizeof(a));
+  a.scale = scale;
+  a.layout = INIT_PLAIN;
+  a.dst = c->embed;
+  a.n_elems = (long long)cf.vocab * d;
+  a.key0 = key(1);
+  DG_CUDA(c, launch_init(a, c->stream));
+  DG_CUDA(c, launch_fill_f32(c->ln_final, d, 1.0f, c->stream));
+  for (int l = 0; l < cf.n_layers; ++l) {
+    Layer& L = c->layers[l];
+    memset(&a, 0, sizeof(a));
+    a.scale = scale;
+    a.layout = INIT_QKV; a.dst = L.wqkv; a.n_elems = (long long)c->NQKV * d;
+    a.key0 = key(ltid(l, 0)); a.key1 = key(ltid(l, 1)); a.key2 = key(ltid(l, 2));
+    a.rows_a = Hq * dh; a.rows_b = Hkv * dh; a.cols = d;
+    DG_CUDA(c, launch_init(a, c->stream));
+    a.layout = INIT_PLAIN; a.dst = L.wo; a.n_elems = (long long)d * Hq * dh; a.key0 = key(ltid(l, 3));
+    DG_CUDA(c, launch_init(a, c->stream));
+    a.dst = L.wr; a.n_elems = (long long)E * d; a.key0 = key(ltid(l, 4));
+    DG_CUDA(c, launch_init(a, c->stream));
+    a.layout = INIT_GATEUP; a.dst = L.wgu; a.n_elems = (long long)c->G * 2 * F * d;
+    a.key0 = key(ltid(l, 5)); a.key1 = key(ltid(l, 6)); a.key2 = key(ltid(l, 8)); a.key3 = key(ltid(l, 9));
+    a.F = F; a.d = d; a.E = E;
+    DG_CUDA(c, launch_init(a, c->stream));
+    a.layout = INIT_DOWN; a.dst = L.wd; a.n_elems = (long long)c->G * d * F;
+    a.key0 = key(ltid(l, 7)); a.key1 = key(ltid(l, 10));
+    DG_CUDA(c, launch_init(a, c->stream));
+    DG_CUDA(c, launch_fill_f32(L.ln_in, d, 1.0f, c->stream));
+    DG_CUDA(c, launch_fill_f32(L.ln_post, d, 1.0f, c->stream));
+    DG_CUDA(c, launch_fill_f32(L.ln_ff, d, 1.0f, c->stream));
+  }
+  DG_CUDA(c, cudaStreamSynchronize(c->stream));
+  c->weights_ready = true;
+  return DG_OK;
+}
+
+int dg_set_prompt_kv(dg_ctx* c, int layer, const void* k, const void* v, int batch, int n_prompt) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= c->cfg.n_layers) return fail(c, DG_ERR_INVALID_ARG, "layer out of range");
+  if (!k || !v) return fail(c, DG_ERR_INVALID_ARG, "null prompt K/V");
+  if (batch < 1 || batch > c->cfg.max_batch) return fail(c, DG_ERR_INVALID_ARG, "batch out of range");
+  if (n_prompt < 1 || n_prompt > c->cfg.max_prompt)
+    return fail(c, DG_ERR_INVALID_ARG, "n_prompt out of range");
+  if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15)
+    return fail(c, DG_ERR_INVALID_ARG, "prompt K/V must be 16-byte aligned");
+  Layer& L = c->layers[layer];
+  L.kp = static_cast<const bf16*>(k);
+  L.vp = static_cast<const bf16*>(v);
+  L.kv_batch = batch;
+  L.kv_P = n_prompt;
+  return DG_OK;
+}
+
+int dg_set_router_bias(dg_ctx* c, const float* bias) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (!bias) { c->has_bias = false; return DG_OK; }
+  DG_CUDA(c, cudaMemcpyAsync(c->router_bias, bias, sizeof(float) * c->cfg.n_experts,
+                             cudaMemcpyDefault, c->stream));
+  c->has_bias = true;
+  return DG_OK;
+}
+
+int dg_canvas_step(dg_ctx* c, int32_t* canvas, int batch, int steps_left, float* conf_out,
+                   uint8_t* committed_out) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (!canvas) return fail(c, DG_ERR_INVALID_ARG, "null canvas");
+  if (batch < 1 || batch > c->cfg.max_batch) return fail(c, DG_ERR_INVALID_ARG, "batch out of range");
+  if (steps_left < 1) return fail(c, DG_ERR_INVALID_ARG, "steps_left must be >= 1");
+  if (!c->weights_ready) return fail(c, DG_ERR_BAD_STATE, "weights not initialised");
+  int rc = check_prompt_state(c, batch);
+  if (rc != DG_OK) return rc;
+  const size_t T = (size_t)batch * c->cfg.canvas_len;
+  DG_CUDA(c, cudaMemcpyAsync(c->canvas_dev, canvas, T * 4, cudaMemcpyDefault, c->stream));
+  if ((rc = run_step(c, batch, steps_left)) != DG_OK) return rc;
+  DG_CUDA(c, cudaMemcpyAsync(canvas, c->canvas_dev, T * 4, cudaMemcpyDefault, c->stream));
+  if (conf_out) DG_CUDA(c, cudaMemcpyAsync(conf_out, c->conf, T * 4, cudaMemcpyDefault, c->stream));
+  if (committed_out)
+    DG_CUDA(c, cudaMemcpyAsync(committed_out, c->committed_dev, T, cudaMemcpyDefault, c->stream));
+  return DG_OK;
+}
+
+int dg_canvas_step_host(dg_ctx* c, int32_t* canvas_host, int batch, int steps_left,
+                        float* conf_host, uint8_t* committed_host) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  int rc = dg_canvas_step(c, canvas_host, batch, steps_left, conf_host, committed_host);
+  if (rc != DG_OK) return rc;
+  DG_CUDA(c, cudaStreamSynchronize(c->stream));
+  return read_device_error(c);
+}
+
+int dg_denoise_block(dg_ctx* c, int32_t* canvas, int batch, int n_steps) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (n_steps < 1) return fail(c, DG_ERR_INVALID_ARG, "n_steps must be >= 1");
+  if (!canvas) return fail(c, DG_ERR_INVALID_ARG, "null canvas");
+  if (batch < 1 || batch > c->cfg.max_batch) return fail(c, DG_ERR_INVALID_ARG, "batch out of range");
+  if (!c->weights_ready) return fail(c, DG_ERR_BAD_STATE, "weights not initialised");
+  int rc = check_prompt_state(c, batch);
+  if (rc != DG_OK) return rc;
+  const size_t T = (size_t)batch * c->cfg.canvas_len;
+  DG_CUDA(c, cudaMemcpyAsync(c->canvas_dev, canvas, T * 4, cudaMemcpyDefault, c->stream));
+  for (int s = 0; s < n_steps; ++s)
+    if ((rc = run_step(c, batch, n_steps - s)) != DG_OK) return rc;
+  DG_CUDA(c, cudaMemcpyAsync(canvas, c->canvas_dev, T * 4, cudaMemcpyDefault, c->stream));
+  return read_device_error(c);
+}
+
+int dg_layer_forward(dg_ctx* c, int layer, const void* x_in, void* x_out, int n_rows) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= c->cfg.n_layers) return fail(c, DG_ERR_INVALID_ARG, "layer out of range");
+  if (!x_in || !x_out) return fail(c, DG_ERR_INVALID_ARG, "null hidden-state pointer");
+  if (!c->weights_ready) return fail(c, DG_ERR_BAD_STATE, "weights not initialised");
+  const Layer& L = c->layers[layer];
+  if (!L.kp) return fail(c, DG_ERR_BAD_STATE, "prompt KV not set for this layer");
+  if (n_rows != L.kv_batch * c->cfg.canvas_len)
+    return fail(c, DG_ERR_INVALID_ARG, "n_rows must equal batch * canvas_len of the prompt KV");
+  const int B = L.kv_batch, d = c->cfg.d_model;
+  int rc;
+  c->launches = 0;
+  if ((rc = ensure_rope(c, L.kv_P)) != DG_OK) return rc;
+  DG_LAUNCH(c, launch_embed_norm(nullptr, nullptr, static_cast<const bf16*>(x_in), c->cfg.vocab,
+                                 n_rows, d, L.ln_in, c->cfg.rms_eps, c->h, c->x, c->err_dev,
+                                 c->stream));
+  if ((rc = run_layer(c, layer, B, nullptr)) != DG_OK) return rc;
+  DG_CUDA(c, cudaMemcpyAsync(x_out, c->x, (size_t)n_rows * d * 2, cudaMemcpyDeviceToDevice,
+                             c->stream));
+  c->last_T = n_rows;
+  c->last_B = B;
+  return DG_OK;
+}
+
+int dg_router_topk(dg_ctx* c, const float* logits, int n_rows, int32_t* idx, float* w,
+                   int32_t* offsets, int32_t* perm) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (!logits || !idx || !w || !offsets || !perm) return fail(c, DG_ERR_INVALID_ARG, "null argument");
+  if (n_rows < 1 || n_rows > c->Tmax) return fail(c, DG_ERR_INVALID_ARG, "n_rows out of range");
+  const int E = c->cfg.n_experts, k = c->cfg.top_k;
+  DG_CUDA(c, launch_router_topk_only(logits, n_rows, E, k, idx, w, c->bitmap, c->stream));
+  DG_CUDA(c, launch_router_sort(idx, c->bitmap, n_rows, E, k, 0, kGroupedTile, offsets, nullptr,
+                                nullptr, perm, c->inv, c->err_dev, c->stream));
+  return DG_OK;
+}
+
+int dg_commit(dg_ctx* c, const float* conf, int32_t* canvas, int batch, int steps_left,
+              const int32_t* cand_tok, uint8_t* committed_out) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (!conf || !canvas || !cand_tok) return fail(c, DG_ERR_INVALID_ARG, "null argument");
+  if (batch < 1 || batch > c->cfg.max_batch) return fail(c, DG_ERR_INVALID_ARG, "batch out of range");
+  if (steps_left < 1) return fail(c, DG_ERR_INVALID_ARG, "steps_left must be >= 1");
+  DG_CUDA(c, launch_commit(conf, cand_tok, canvas, committed_out, batch, c->cfg.canvas_len,
+                           steps_left, nullptr, c->cfg.mask_id, c->stream));
+  return DG_OK;
+}
+
+int dg_debug_tensor(dg_ctx* c, const char* name, void* dst, size_t bytes, size_t* bytes_needed) {
+  if (!c || !name) return DG_ERR_INVALID_ARG;
+  const dg_config& cf = c->cfg;
+  const size_t T = c->last_T, d = cf.d_model, E = cf.n_experts, k = cf.top_k;
+  const size_t dh = cf.head_dim, Hq = cf.n_q_heads, Hkv = cf.n_kv_heads;
+  const void* src = nullptr;
+  size_t n = 0;
+  const std::string s(name);
+  if (s == "x" || s == "hn") { src = c->x; n = T * d * 2; }
+  else if (s == "q") { src = c->q; n = T * Hq * dh * 2; }
+  else if (s == "kc") { src = c->kc; n = T * Hkv * dh * 2; }
+  else if (s == "vc") { src = c->vc; n = T * Hkv * dh * 2; }
+  else if (s == "attn_o") { src = c->attn_o; n = T * Hq * dh * 2; }
+  else if (s == "h") { src = c->h; n = T * d * 4; }
+  else if (s == "x2") { src = c->xperm; n = T * d * 2; }
+  else if (s == "router_logits") { src = c->router_logits; n = T * E * 4; }
+  else if (s == "idx") { src = c->idx; n = T * k * 4; }
+  else if (s == "w") { src = c->w; n = T * k * 4; }
+  else if (s == "offsets") { src = c->offsets_r; n = (E + 1) * 4; }
+  else if (s == "perm") { src = c->perm; n = T * k * 4; }
+  else if (s == "tok") { src = c->tok; n = T * 4; }
+  else if (s == "conf") { src = c->conf; n = T * 4; }
+  else if (s == "embed") { src = c->embed; n = (size_t)cf.vocab * d * 2; }
+  else {
+    // weights of one layer: "<name>:<layer>"
+    const size_t colon = s.find(':');
+    if (colon == std::string::npos) return fail(c, DG_ERR_INVALID_ARG, "unknown tensor name");
+    const std::string base = s.substr(0, colon);
+    const int l = std::atoi(s.c_str() + colon + 1);
+    if (l < 0 || l >= cf.n_layers) return fail(c, DG_ERR_INVALID_ARG, "layer out of range");
+    const Layer& L = c->layers[l];
+    const size_t F = cf.d_ff;
+    if (base == "wqkv") { src = L.wqkv; n = (size_t)c->NQKV * d * 2; }
+    else if (base == "wo") { src = L.wo; n = d * Hq * dh * 2; }
+    else if (base == "wr") { src = L.wr; n = E * d * 2; }
+    else if (base == "wgu") { src = L.wgu; n = (size_t)c->G * 2 * F * d * 2; }
+    else if (base == "wd") { src = L.wd; n = (size_t)c->G * d * F * 2; }
+    else return fail(c, DG_ERR_INVALID_ARG, "unknown tensor name");
+  }
+  if (bytes_needed) *bytes_needed = n;
+  if (!dst) return DG_OK;
+  if (bytes < n) return fail(c, DG_ERR_INVALID_ARG, "destination too small");
+  DG_CUDA(c, cudaMemcpyAsync(dst, src, n, cudaMemcpyDefault, c->stream));
+  DG_CUDA(c, cudaStreamSynchronize(c->stream));
+  return DG_OK;
+}
+
+int dg_sync(dg_ctx* c) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  DG_CUDA(c, cudaStreamSynchronize(c->stream));
+  return read_device_error(c);
+}
+
+const char* dg_last_error(const dg_ctx* c) {
+  return c ? c->err.c_str() : g_create_error.c_str();
+}
+
+size_t dg_device_bytes(const dg_ctx* c) { return c ? c->bytes : 0; }
+
+int dg_last_launch_count(const dg_ctx* c) { return c ? c->launches : 0; }
+
+void dg_destroy(dg_ctx* c) {
+  if (!c) return;
+  cudaStreamSynchronize(c->stream);
+  free_all(c);
+  delete c;
+}
+
+}  // extern "C"

@@ -1,0 +1,137 @@
+// Internal kernel interfaces of libdg (not part of the C ABI).
+#pragma once
+
+#include "dg_common.cuh"
+
+namespace dg {
+
+enum GemmMode { GEMM_DENSE = 0, GEMM_GATEUP = 1, GEMM_DOWN = 2, GEMM_HEAD = 3 };
+
+struct GemmArgs {
+  int mode;
+  int M, N, K, n_kb;      // A rows, B rows, reduction length, K / 64
+  int n_tile;             // B rows per tile (DENSE / grouped)
+  int k_splits;           // DENSE split-K
+  int m_slabs;            // 128-row slabs of A per group (DENSE / grouped)
+  int n_groups;           // grouped: number of groups
+  const int* offsets;     // grouped: [n_groups + 1] first B row of each group
+  const int* chunk_prefix;// grouped: [n_groups + 1] prefix of ceil(rows_g / n_tile)
+  int F;                  // GATEUP output width
+  int T, vocab, mask_id;  // HEAD
+  int n_vblocks, n_tblocks;
+  float* out_f32;
+  bf16* out_bf16;
+  float* head_m;
+  float* head_s;
+  int* head_a;
+  int* err;
+  // shared-memory plan (gemm_plan_smem)
+  int stages, a_bytes, b_bytes, stage_bytes, b_box_rows;
+};
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                  uint32_t box_outer);
+bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid,
+                  uint64_t outer, uint32_t box_mid);
+void gemm_plan_smem(GemmArgs& a);
+size_t gemm_smem_bytes(const GemmArgs& a);
+cudaError_t gemm_tc_launch(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmArgs& a,
+                           int grid, cudaStream_t stream);
+
+// ---------------------------------------------------------------- weight init
+// Physical layouts of the generated tensors (see init kernels).
+enum InitLayout {
+  INIT_PLAIN = 0,   // physical == logical [rows][cols] of tensor tid
+  INIT_QKV = 1,     // rows [0,nq) tid_q, [nq,nq+nkv) tid_k, rest tid_v; cols d
+  INIT_GATEUP = 2,  // [E+1][2F][d]: group 0 shared expert, group g>0 expert g-1;
+                    // row 2f = gate row f, row 2f+1 = up row f
+  INIT_DOWN = 3     // [E+1][d][F]: group 0 shared expert, group g>0 expert g-1
+};
+
+struct InitArgs {
+  int layout;
+  bf16* dst;
+  long long n_elems;     // physical elements
+  unsigned long long key0, key1, key2, key3;  // stream keys (meaning per layout)
+  int rows_a, rows_b;    // QKV: nq, nkv
+  int cols;              // innermost width (d or F)
+  int F, d, E;           // grouped layouts
+  float scale;           // float32(std * sqrt(3) / 65536)
+};
+
+unsigned long long stream_key_host(unsigned long long seed, unsigned long long tid);
+cudaError_t launch_init(const InitArgs& a, cudaStream_t s);
+cudaError_t launch_fill_f32(float* p, long long n, float v, cudaStream_t s);
+
+// ---------------------------------------------------------------- elementwise / norm
+// h[t] = float(E[canvas[t]]) (or float(x_in[t]) when x_in != NULL);
+// x[t] = bf16(rmsnorm(h[t]) * w)
+cudaError_t launch_embed_norm(const int32_t* canvas, const bf16* embed, const bf16* x_in,
+                              int vocab, int T, int d, const float* w, float eps, float* h,
+                              bf16* x, int* err, cudaStream_t s);
+
+// cos/sin table [Tc][dh/2] for positions P + i, in double precision.
+cudaError_t launch_rope_table(float* cos_t, float* sin_t, int Tc, int half, int P, double theta,
+                              cudaStream_t s);
+
+// Sum QKV split-K partials, rotate q and k (first n_rot pairs), scatter to
+// q [B][Hq][Tc][dh], kc/vc [B][Hkv][Tc][dh] (bf16).
+cudaError_t launch_qkv_rope(const float* part, int splits, int T, int Tc, int Hq, int Hkv, int dh,
+                            int n_rot, const float* cos_t, const float* sin_t, bf16* q, bf16* kc,
+                            bf16* vc, cudaStream_t s);
+
+struct AttnArgs {
+  const bf16* q;   // [B][Hq][Tc][dh]
+  const bf16* kc;  // [B][Hkv][Tc][dh]
+  const bf16* vc;
+  const bf16* kp;  // [B][Hkv][P][dh]
+  const bf16* vp;
+  int B, Hq, Hkv, Tc, P, dh;
+  int n_vis;       // visible prompt keys (the last n_vis)
+  int n_chunks, chunk_keys;
+  float* part_o;   // [n_chunks][B*Hq*Tc][dh]
+  float* part_ml;  // [n_chunks][B*Hq*Tc][2]  (max in log2 units, sum)
+  float scale_log2;  // log2(e) / sqrt(dh)
+};
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
+// Merge partials -> o [T][Hq*dh] bf16 (t = b*Tc + i)
+cudaError_t launch_attn_merge(const AttnArgs& a, bf16* o, cudaStream_t s);
+
+// a = sum of O-projection partials; h1 = h + rmsnorm(a)*w_post (h updated in
+// place); x2 = bf16(rmsnorm(h1)*w_ff).
+cudaError_t launch_post_attn(const float* part, int splits, int T, int d, const float* w_post,
+                             const float* w_ff, float eps, float* h, bf16* x2, cudaStream_t s);
+
+// Router: logits = sum partials (+bias); top-k; weights; bitmap of expert membership.
+cudaError_t launch_router_topk(const float* part, int splits, const float* bias, int T, int E,
+                               int k, float* logits_out, int32_t* idx, float* w,
+                               uint32_t* bitmap, cudaStream_t s);
+// Counting sort (single CTA).  Routed offsets_r [E+1] and perm/inv [T*k] are
+// relative to the routed block; offsets_g / chunk_prefix [E+2] describe the
+// grouped-GEMM groups: group 0 = shared expert rows [0, T), group e+1 =
+// expert e rows [T + offsets_r[e], T + offsets_r[e+1]).  Clears the bitmap.
+cudaError_t launch_router_sort(const int32_t* idx, uint32_t* bitmap, int T, int E, int k,
+                               int n_shared, int n_tile, int32_t* offsets_r, int32_t* offsets_g,
+                               int32_t* chunk_prefix, int32_t* perm, int32_t* inv, int* err,
+                               cudaStream_t s);
+// xperm[T + p] = xperm[perm[p] / k] for p < k*T (rows [0, T) hold the normed input).
+cudaError_t launch_moe_gather(bf16* xperm, const int32_t* perm, int T, int k, int d,
+                              cudaStream_t s);
+// h = h + sum_j w[t][j] Y[T + inv[t*k+j]] (+ Y[t] shared); then either
+// x = bf16(rmsnorm(h)*w_next) (w_next != NULL) or x = bf16(h).
+cudaError_t launch_moe_combine(const float* Y, const float* w, const int32_t* inv, int T, int k,
+                               int n_shared, int d, float* h, const float* w_next, float eps,
+                               bf16* x, cudaStream_t s);
+
+// Vocab head merge over vocab blocks: conf = 1/sum, tok = argmax.
+cudaError_t launch_head_merge(const float* hm, const float* hs, const int* ha, int n_vblocks,
+                              int T, float* conf, int32_t* tok, cudaStream_t s);
+// Commit (one block per canvas).  steps_left read from *steps_left_dev when
+// steps_left < 0.
+cudaError_t launch_commit(const float* conf, const int32_t* tok, int32_t* canvas,
+                          uint8_t* committed, int B, int Tc, int steps_left,
+                          const int* steps_left_dev, int mask_id, cudaStream_t s);
+cudaError_t launch_router_topk_only(const float* logits, int T, int E, int k, int32_t* idx,
+                                    float* w, uint32_t* bitmap, cudaStream_t s);
+
+}  // namespace dg

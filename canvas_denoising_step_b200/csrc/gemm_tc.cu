@@ -1,0 +1,399 @@
+// Persistent, warp-specialised tcgen05 GEMM for sm_100a.
+//
+// Roles (192 threads): warp 0 lane 0 issues TMA loads into a ring of shared
+// memory stages; warp 1 lane 0 issues tcgen05.mma into TMEM accumulators
+// (warp 1 also allocates TMEM); warps 2..5 are the epilogue, each reading its
+// 32-lane quadrant of TMEM with tcgen05.ld.  Accumulators are double
+// buffered so the epilogue of one tile overlaps the MMAs of the next.
+//
+// Operands are K-major bf16 tiles with the 128-byte swizzle (64 elements of
+// K per row).  The MMA is always M = 128: "A" rows are the output features
+// for the weight-streaming modes (the weight is the M operand, the few
+// activation rows are N), and the token rows for the vocab head.
+//
+// Modes
+//  DENSE   Y[s][n][m] = sum_{k in split s} X[n][k] W[m][k]      (fp32 split-K partials)
+//  GATEUP  H[r][f] = silu(g) * u, with g/u the gate/up rows 2f/2f+1 of the
+//          group's interleaved weight, for rows r of the group     (bf16)
+//  DOWN    Y[r][m] = sum_k H[r][k] Wd[g][m][k]                   (fp32)
+//  HEAD    per token row t and 256-wide vocab block b: the max logit, its
+//          index (lowest on ties) and sum exp(l - max) over the block, with
+//          the mask id and out-of-range vocab rows excluded      (partials)
+#include "dg_kernels.h"
+
+namespace dg {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kBK = 64;             // K elements per stage (128-byte rows)
+constexpr int kATileBytes = 128 * 128;  // 128 rows x 128 B
+
+struct TileInfo {
+  int g, m_slab, row0, rows, kb0, kb1, split, tb, vb;
+  int n_acc;   // accumulators (A tiles) per tile
+  int n_mma;   // MMA N
+  int n_bbox;  // B boxes per stage
+};
+
+__device__ __forceinline__ int upper_bound_prefix(const int* prefix, int n, int c) {
+  // largest g in [0, n) with prefix[g] <= c
+  int lo = 0, hi = n;  // prefix[0] == 0 <= c
+  while (hi - lo > 1) {
+    int mid = (lo + hi) >> 1;
+    if (__ldg(prefix + mid) <= c) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ int tile_count(const GemmArgs& a) {
+  switch (a.mode) {
+    case GEMM_DENSE: return a.m_slabs * ((a.N + a.n_tile - 1) / a.n_tile) * a.k_splits;
+    case GEMM_GATEUP:
+    case GEMM_DOWN: return __ldg(a.chunk_prefix + a.n_groups) * a.m_slabs;
+    default: return a.n_vblocks * a.n_tblocks;
+  }
+}
+
+__device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t) {
+  TileInfo ti;
+  ti.g = 0; ti.split = 0; ti.tb = 0; ti.vb = 0; ti.n_acc = 1;
+  if (a.mode == GEMM_DENSE) {
+    const int n_chunks = (a.N + a.n_tile - 1) / a.n_tile;
+    ti.m_slab = t % a.m_slabs;
+    const int rest = t / a.m_slabs;
+    const int chunk = rest % n_chunks;
+    ti.split = rest / n_chunks;
+    ti.row0 = chunk * a.n_tile;
+    ti.rows = min(a.n_tile, a.N - ti.row0);
+    ti.kb0 = (int)(((long long)ti.split * a.n_kb) / a.k_splits);
+    ti.kb1 = (int)(((long long)(ti.split + 1) * a.n_kb) / a.k_splits);
+  } else if (a.mode == GEMM_GATEUP || a.mode == GEMM_DOWN) {
+    ti.m_slab = t % a.m_slabs;
+    const int c = t / a.m_slabs;
+    ti.g = upper_bound_prefix(a.chunk_prefix, a.n_groups, c);
+    const int j = c - __ldg(a.chunk_prefix + ti.g);
+    const int beg = __ldg(a.offsets + ti.g), end = __ldg(a.offsets + ti.g + 1);
+    ti.row0 = beg + j * a.n_tile;
+    ti.rows = min(a.n_tile, end - ti.row0);
+    ti.kb0 = 0;
+    ti.kb1 = a.n_kb;
+  } else {  // HEAD
+    ti.tb = t % a.n_tblocks;
+    ti.vb = t / a.n_tblocks;
+    ti.m_slab = 0;
+    ti.row0 = ti.vb * 256;
+    ti.rows = 256;
+    ti.n_acc = (a.T - ti.tb * 256 > 128) ? 2 : 1;
+    ti.kb0 = 0;
+    ti.kb1 = a.n_kb;
+  }
+  if (a.mode == GEMM_HEAD) {
+    ti.n_mma = 256;
+    ti.n_bbox = 1;
+  } else {
+    ti.n_mma = (ti.rows + 15) & ~15;
+    ti.n_bbox = (ti.rows + a.b_box_rows - 1) / a.b_box_rows;
+  }
+  return ti;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+               const GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int S = a.stages;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * a.stage_bytes);
+  // full[0..S), empty[S..2S), tmem_full[2S..2S+2), tmem_empty[2S+2..2S+4)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t smem_base = smem_u32(smem);
+  const uint32_t bar_base = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (S + s); };
+  auto tfull_bar = [&](int b) { return bar_base + 8u * (2 * S + b); };
+  auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * S + 2 + b); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&mapA);
+    tma_prefetch_desc(&mapB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int n_tiles = tile_count(a);
+  const int n_bufs = (a.mode == GEMM_HEAD) ? 1 : 2;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      bool wrapped = false, ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const TileInfo ti = decode_tile(a, t);
+        const uint32_t tx = (uint32_t)(ti.n_acc * kATileBytes) +
+                            (uint32_t)(ti.n_bbox * a.b_box_rows * 128);
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.err)) { ok = false; break; }
+          const uint32_t sA = smem_base + (uint32_t)stage * a.stage_bytes;
+          const uint32_t sB = sA + (uint32_t)a.a_bytes;
+          const uint32_t fb = full_bar(stage);
+          mbar_arrive_expect_tx(fb, tx);
+          const int kx = kb * kBK;
+          if (a.mode == GEMM_DENSE) {
+            tma_load_2d(sA, &mapA, fb, kx, ti.m_slab * 128);
+          } else if (a.mode == GEMM_HEAD) {
+            for (int i = 0; i < ti.n_acc; ++i)
+              tma_load_2d(sA + i * kATileBytes, &mapA, fb, kx, ti.tb * 256 + i * 128);
+          } else {
+            tma_load_3d(sA, &mapA, fb, kx, ti.m_slab * 128, ti.g);
+          }
+          for (int i = 0; i < ti.n_bbox; ++i)
+            tma_load_2d(sB + (uint32_t)(i * a.b_box_rows * 128), &mapB, fb, kx,
+                        ti.row0 + i * a.b_box_rows);
+          if (++stage == S) { stage = 0; phase ^= 1u; wrapped = true; }
+        }
+      }
+      if (!ok) {  // abort path: let issued copies land before the CTA exits
+        for (int s = 0; s < S; ++s) {
+          if (s < stage) mbar_drain(full_bar(s), phase);
+          else if (wrapped) mbar_drain(full_bar(s), phase ^ 1u);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
+        const TileInfo ti = decode_tile(a, t);
+        const int buf = it % n_bufs;
+        const uint32_t tph = (uint32_t)((it / n_bufs) & 1);
+        if (!mbar_wait(tempty_bar(buf), tph ^ 1u, abort_flag, a.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_base = tmem_base + (uint32_t)buf * 256u;
+        const uint32_t idesc = idesc_bf16_f32(ti.n_mma);
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, a.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sA = smem_base + (uint32_t)stage * a.stage_bytes;
+          const uint32_t sB = sA + (uint32_t)a.a_bytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t bdesc = sdesc_kmajor_sw128(sB + kk * 32);
+            for (int i = 0; i < ti.n_acc; ++i) {
+              const uint64_t adesc = sdesc_kmajor_sw128(sA + i * kATileBytes + kk * 32);
+              umma_bf16(d_base + (uint32_t)i * 256u, adesc, bdesc, idesc,
+                        (kb > ti.kb0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(empty_bar(stage));
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(tfull_bar(buf));
+      }
+    }
+    __syncwarp();
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int q = warp & 3;                 // TMEM lane quadrant of this warp
+    const int r = q * 32 + lane;            // accumulator row (TMEM lane)
+    int it = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
+      const TileInfo ti = decode_tile(a, t);
+      const int buf = it % n_bufs;
+      const uint32_t tph = (uint32_t)((it / n_bufs) & 1);
+      if (!mbar_wait(tfull_bar(buf), tph, abort_flag, a.err)) break;
+      tc_fence_after();
+      const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)buf * 256u;
+      uint32_t v[32];
+      if (a.mode == GEMM_DENSE || a.mode == GEMM_DOWN) {
+        const int m = ti.m_slab * 128 + r;
+        float* out = a.out_f32 + (size_t)ti.split * a.N * a.M;
+        for (int c0 = 0; c0 < ti.n_mma; c0 += 32) {
+          tmem_ld32(lane_addr + c0, v);
+          tmem_wait_ld();
+          if (m < a.M) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int n = c0 + j;
+              if (n < ti.rows) out[(size_t)(ti.row0 + n) * a.M + m] = __uint_as_float(v[j]);
+            }
+          }
+        }
+      } else if (a.mode == GEMM_GATEUP) {
+        // Interleaved rows: even accumulator rows are gate rows, odd rows the
+        // matching up rows of the same output feature f.
+        const int f = (ti.m_slab * 128 + r) >> 1;
+        const bool is_gate = (r & 1) == 0;
+        for (int c0 = 0; c0 < ti.n_mma; c0 += 32) {
+          tmem_ld32(lane_addr + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float x = __uint_as_float(v[j]);
+            const float u = __shfl_xor_sync(0xffffffffu, x, 1);
+            const int n = c0 + j;
+            if (is_gate && n < ti.rows && f < a.F) {
+              const float h = x / (1.0f + __expf(-x)) * u;
+              a.out_bf16[(size_t)(ti.row0 + n) * a.F + f] = f_to_bf16(h);
+            }
+          }
+        }
+      } else {  // HEAD
+        for (int i = 0; i < ti.n_acc; ++i) {
+          const int tok_row = ti.tb * 256 + i * 128 + r;
+          float mx = -INFINITY, sum = 0.f;
+          int arg = -1;
+          for (int c0 = 0; c0 < 256; c0 += 32) {
+            tmem_ld32(lane_addr + (uint32_t)i * 256u + c0, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int vid = ti.row0 + c0 + j;
+              if (vid < a.vocab && vid != a.mask_id) {
+                const float x = __uint_as_float(v[j]);
+                if (x > mx) {
+                  sum = sum * __expf(mx - x) + 1.0f;
+                  mx = x;
+                  arg = vid;
+                } else {
+                  sum += __expf(x - mx);
+                }
+              }
+            }
+          }
+          if (tok_row < a.T) {
+            const size_t o = (size_t)ti.vb * a.T + tok_row;
+            a.head_m[o] = mx;
+            a.head_s[o] = sum;
+            a.head_a[o] = arg;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(buf));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ============================================================================ host side
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                  uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid,
+                  uint64_t outer, uint32_t box_mid) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, mid, outer};
+  cuuint64_t strides[2] = {inner * 2, inner * mid * 2};
+  cuuint32_t box[3] = {64, box_mid, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Shared-memory plan: A region (1 or 2 tiles of 16 KB) + B region, as many
+// stages as fit in ~220 KB.
+void gemm_plan_smem(GemmArgs& a) {
+  const int n_a = (a.mode == GEMM_HEAD) ? 2 : 1;
+  a.a_bytes = n_a * kATileBytes;
+  if (a.mode == GEMM_HEAD) {
+    a.b_box_rows = 256;
+    a.b_bytes = 256 * 128;
+  } else {
+    a.b_box_rows = 32;
+    a.b_bytes = ((a.n_tile + 31) / 32) * 32 * 128;
+  }
+  a.stage_bytes = a.a_bytes + a.b_bytes;  // multiples of 1024
+  int s = (220 * 1024) / a.stage_bytes;
+  a.stages = s < 2 ? 2 : (s > 8 ? 8 : s);
+}
+
+size_t gemm_smem_bytes(const GemmArgs& a) {
+  return 1024 + (size_t)a.stages * a.stage_bytes + (2 * a.stages + 4) * 8 + 16;
+}
+
+cudaError_t gemm_tc_launch(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmArgs& a,
+                           int grid, cudaStream_t stream) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  gemm_tc_kernel<<<grid, kThreads, gemm_smem_bytes(a), stream>>>(mapA, mapB, a);
+  return cudaGetLastError();
+}
+
+}  // namespace dg

@@ -1,0 +1,219 @@
+/*
+ * dg.h -- C ABI of the B200 (sm_100a) canvas denoising step library (libdg.so).
+ *
+ * The operation: a canvas of canvas_len token slots (256 on the pages) that
+ * starts as all [MASK] is refined by repeated passes through a stack of
+ * decoder blocks; each pass ends by locking in the most confident
+ * still-masked slots.  Sources (page title, section):
+ *   "Hands-On with Diffusion Gemma: Another Gemma with a Diffusion Mechanism",
+ *     "How Is This Different from Previous Models?" (canvas of 256 masked
+ *     slots, repeated decoding passes) and "Detailed Specs" (30 blocks as
+ *     (5 local + 1 global) x 5, hidden 2816, MoE, sliding-window local
+ *     attention, GQA global attention, RoPE / p-RoPE, tied embed_tokens and
+ *     lm_head, input / post-attention / pre-feedforward / final norms,
+ *     router, encoder KV cache shared with the decoder);
+ *   "DiffusionGemma: The Diffusion Era Begins with 4x Faster Text Generation",
+ *     "What is Diffusion ..." (locked tokens become context) and
+ *     "DiffusionGemma's Technical Architecture" (128 experts, 8 active + 1
+ *     shared, canvas 256, window 1024, vocab 262K, bidirectional attention
+ *     over the canvas plus cross-attention into the prompt's cached KV);
+ *   "DiffusionGemma: Google's Experimental Diffusion LLM", "How Text
+ *     Diffusion Actually Works" (a small fixed number of passes per block).
+ * Readings where the pages are silent (one joint softmax over prompt window
+ * and canvas, RMSNorm with unit scales, p = 0.25 for p-RoPE, top-k by logit
+ * with lowest-index ties, k = ceil(remaining / steps_left) commits per pass,
+ * confidence = largest softmax probability with the mask id excluded) are the
+ * library's defined behaviour; each is stated at the call it affects.
+ *
+ * Conventions for every call:
+ *  - Return value: DG_OK (0) or a negative DG_ERR_* code.  No C++ exception
+ *    crosses this interface.  dg_last_error() gives a text for the last error
+ *    of a context.
+ *  - Argument errors are detected before any work is queued and leave every
+ *    output untouched.
+ *  - All work is queued on the CUDA stream given to dg_create() and is
+ *    asynchronous unless stated otherwise.  A context is not thread-safe.
+ *  - Errors raised inside kernels (a bounded wait that gave up, an index out
+ *    of range) are recorded in a device error word and reported by dg_sync()
+ *    (and by the calls that end with a synchronisation).
+ *  - "dev" pointers are CUDA device pointers, "host" pointers ordinary host
+ *    memory.  The library never frees a caller's pointer.
+ *  - Matrices are row-major.  bf16 is IEEE bfloat16 stored as uint16_t.
+ */
+#ifndef DG_H
+#define DG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  DG_OK = 0,
+  DG_ERR_INVALID_ARG = -1,   /* a null pointer, a size out of range, a bad config */
+  DG_ERR_BAD_STATE = -2,     /* call out of order (e.g. a step before the prompt KV is set) */
+  DG_ERR_OOM = -3,           /* a device allocation failed or would pass alloc_limit_bytes */
+  DG_ERR_CUDA = -4,          /* a CUDA runtime call failed (no device, launch failure) */
+  DG_ERR_TIMEOUT = -5,       /* a bounded in-kernel wait gave up; results are invalid */
+  DG_ERR_DEVICE_FAULT = -6,  /* a kernel flagged an out-of-range index; results are invalid */
+  DG_ERR_UNSUPPORTED = -7    /* a shape outside what the kernels implement */
+};
+
+typedef struct dg_ctx dg_ctx;
+
+/*
+ * Model and capacity description.  Shape limits checked by dg_create():
+ *   d_model a multiple of 64 in [128, 4096]; d_ff a multiple of 64;
+ *   head_dim in {64, 128, 256};
+ *   n_q_heads a multiple of n_kv_heads; 1 <= top_k <= min(n_experts, 32);
+ *   n_experts <= 256;
+ *   n_shared in {0, 1}; 1 <= canvas_len <= 256; max_batch * canvas_len <= 4096;
+ *   0 <= mask_id < vocab; window >= 1; global_every >= 1.
+ * Layer l (0-based) is global iff (l + 1) % global_every == 0: it attends to
+ * all prompt keys and rotates the first ceil(prope_fraction * head_dim / 2)
+ * RoPE pairs.  Other layers attend to the last min(window, n_prompt) prompt
+ * keys and rotate every pair.  rope_enabled = 0 turns all rotation off.
+ * weight_std is the standard deviation of the seeded weights (0.02).
+ */
+typedef struct dg_config {
+  int n_layers, d_model, n_q_heads, n_kv_heads, head_dim;
+  int n_experts, top_k, n_shared, d_ff;
+  int vocab, canvas_len, window, global_every;
+  int mask_id, max_batch, max_prompt;
+  float rms_eps, rope_theta, prope_fraction;
+  int rope_enabled;
+  double weight_std;         /* the generator's scale is float32(weight_std * sqrt(3) / 65536) */
+  size_t alloc_limit_bytes;  /* 0 = no limit; otherwise dg_create fails with DG_ERR_OOM
+                                instead of allocating more than this many device bytes */
+} dg_config;
+
+/* Creates a context on the current CUDA device: checks the config, allocates
+ * the weights (bf16) and the workspace, and records `cuda_stream`
+ * (a cudaStream_t, NULL = legacy default stream).  Weights are not yet drawn.
+ * *out is set only on success.  Synchronous. */
+int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out);
+
+/* Draws every weight on the device from `seed` (the tied embedding, and per
+ * layer the q/k/v/o projections, router, routed experts' gate/up/down and the
+ * shared expert's gate/up/down), N(0, weight_std) by the SplitMix64 counter
+ * generator with a four-term Irwin-Hall normal, rounded to bf16; norm scales
+ * are set to 1.  The value of each logical element depends only on
+ * (seed, tensor, element index), never on the physical layout. */
+int dg_init_weights(dg_ctx* ctx, uint64_t seed);
+
+/* Borrows the prompt's cached keys and values for one layer (the encoder's KV
+ * cache the decoder cross-attends to).  k, v: dev bf16 [batch][n_kv_heads]
+ * [n_prompt][head_dim], keys already rotated.  No copy is made: the buffers
+ * must stay valid and unchanged until this layer's next dg_set_prompt_kv or
+ * dg_destroy.  Every layer must be given the same batch and n_prompt before a
+ * step; canvas row i then sits at position n_prompt + i.
+ * 1 <= batch <= max_batch, 1 <= n_prompt <= max_prompt. */
+int dg_set_prompt_kv(dg_ctx* ctx, int layer, const void* k, const void* v,
+                     int batch, int n_prompt);
+
+/* Adds a fixed bias (dev fp32 [n_experts]) to the router logits of every
+ * layer, or removes it when bias == NULL.  The bias is copied. */
+int dg_set_router_bias(dg_ctx* ctx, const float* bias);
+
+/* One denoising pass over `batch` canvases, then the commit.
+ * canvas: dev int32 [batch][canvas_len], updated in place: with r the number
+ * of slots equal to mask_id in a canvas, the k = ceil(r / steps_left) masked
+ * slots of highest confidence (ties toward the lower slot) receive their
+ * argmax token; all other slots are unchanged.  steps_left >= 1.
+ * conf_out (dev fp32 [batch][canvas_len]) receives every slot's confidence,
+ * the largest softmax probability of its logits with the mask id excluded;
+ * committed_out (dev uint8 [batch][canvas_len]) receives 1 for the slots
+ * committed by this pass.  Both may be NULL. */
+int dg_canvas_step(dg_ctx* ctx, int32_t* canvas, int batch, int steps_left,
+                   float* conf_out, uint8_t* committed_out);
+
+/* dg_canvas_step on HOST buffers: copies the canvas to the device, runs the
+ * pass, copies canvas (and conf / committed when not NULL) back, and returns
+ * after the results are in host memory (synchronous). */
+int dg_canvas_step_host(dg_ctx* ctx, int32_t* canvas_host, int batch, int steps_left,
+                        float* conf_host, uint8_t* committed_host);
+
+/* n_steps passes with steps_left = n_steps, n_steps - 1, ..., 1: every masked
+ * slot is committed at the end.  canvas: dev int32 [batch][canvas_len], in
+ * place.  Ends with a synchronisation and reports device errors. */
+int dg_denoise_block(dg_ctx* ctx, int32_t* canvas, int batch, int n_steps);
+
+/* One decoder block on given hidden states (no embedding, head or commit):
+ * x_out = block(x_in) with x_in, x_out dev bf16 [n_rows][d_model],
+ * n_rows = batch * canvas_len for the batch given to dg_set_prompt_kv.
+ * x_in and x_out may be the same buffer. */
+int dg_layer_forward(dg_ctx* ctx, int layer, const void* x_in, void* x_out, int n_rows);
+
+/* Router test hook: top_k selection and grouping from given logits.
+ * logits: dev fp32 [n_rows][n_experts] (used as given; the router bias is not
+ * added).  Outputs (dev): idx int32 [n_rows][top_k], experts by decreasing
+ * logit, equal logits toward the lower index; w fp32 [n_rows][top_k], the
+ * softmax over the chosen logits; offsets int32 [n_experts + 1]; perm int32
+ * [n_rows * top_k] with perm[offsets[e] + r] = t * top_k + j for the r-th
+ * assignment (t, j) to expert e in increasing t.  n_rows <= max_batch *
+ * canvas_len. */
+int dg_router_topk(dg_ctx* ctx, const float* logits, int n_rows, int32_t* idx, float* w,
+                   int32_t* offsets, int32_t* perm);
+
+/* Commit test hook: the commit rule of dg_canvas_step on given confidences.
+ * conf: dev fp32 [batch][canvas_len]; cand_tok: dev int32 [batch][canvas_len]
+ * (the token each slot would receive); canvas: dev int32, in place;
+ * committed_out: dev uint8 or NULL. */
+int dg_commit(dg_ctx* ctx, const float* conf, int32_t* canvas, int batch, int steps_left,
+              const int32_t* cand_tok, uint8_t* committed_out);
+
+/* Debug hook: copies an internal tensor of the most recent pass (or layer
+ * call) into dst (dev or host, `bytes` long; cudaMemcpyDefault), synchronously.
+ * *bytes_needed (may be NULL) receives the tensor's size; with dst == NULL
+ * only the size is reported.  Names and contents:
+ *   "x"        bf16 [T][d]        after dg_layer_forward: the block output; after a
+ *                                 pass: the final-normed states fed to the vocab head
+ *   "hn"       the same buffer as "x"
+ *   "q"        bf16 [B][Hq][Tc][dh]   rotated queries; "kc", "vc" likewise [B][Hkv][Tc][dh]
+ *                                 (rotated canvas keys, canvas values) of the last layer run
+ *   "attn_o"   bf16 [T][Hq*dh]    attention output before the output projection
+ *   "x2"       bf16 [T][d]        pre-feedforward-normed hidden states
+ *   "router_logits" fp32 [T][E]   (bias included)
+ *   "idx" int32 [T][k]; "w" fp32 [T][k]; "offsets" int32 [E+1]; "perm" int32 [T*k]
+ *                                 (the routing of the last layer run, as dg_router_topk)
+ *   "h"        fp32 [T][d]        residual stream after the last layer run
+ *   "tok"      int32 [T]          argmax token per row (after a pass)
+ *   "conf"     fp32 [T]           confidence per row (after a pass)
+ * and the weights (bf16, physical layouts):
+ *   "embed"    [vocab][d]
+ *   "wqkv:L"   [(Hq+2Hkv)*dh][d]  rows: q heads, then k heads, then v heads
+ *   "wo:L"     [d][Hq*dh];  "wr:L" [E][d]
+ *   "wgu:L"    [E+1][2*d_ff][d]   group 0 = shared expert, group g = expert g-1;
+ *                                 row 2f = gate row f, row 2f+1 = up row f
+ *   "wd:L"     [E+1][d][d_ff]     group 0 = shared expert, group g = expert g-1
+ * with T = batch * canvas_len rows of the last call. */
+int dg_debug_tensor(dg_ctx* ctx, const char* name, void* dst, size_t bytes,
+                    size_t* bytes_needed);
+
+/* Waits for the context's stream and reports (then clears) the device error
+ * word: DG_ERR_TIMEOUT or DG_ERR_DEVICE_FAULT if a kernel raised one. */
+int dg_sync(dg_ctx* ctx);
+
+/* Text of the context's last error ("" if none).  With ctx == NULL, the text
+ * of the last error of a dg_create that returned no context.  The pointer
+ * stays valid until the next call on the same context. */
+const char* dg_last_error(const dg_ctx* ctx);
+
+/* Device bytes held by the context (weights + workspace). */
+size_t dg_device_bytes(const dg_ctx* ctx);
+
+/* Kernel launches queued by the most recent dg_canvas_step /
+ * dg_layer_forward (for launch accounting). */
+int dg_last_launch_count(const dg_ctx* ctx);
+
+/* Frees everything the context owns (not the borrowed prompt K/V).
+ * Synchronises the stream first.  NULL is ignored. */
+void dg_destroy(dg_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_H */

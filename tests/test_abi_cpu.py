@@ -1,0 +1,94 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/dg.h declares, its config struct matches the binding's mirror, and
+argument / no-device errors come back as status codes."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dg.h")
+
+
+@pytest.fixture(scope="module")
+def dg():
+    from canvas_denoising_step_b200.build import build
+    build()
+    import canvas_denoising_step_b200 as m
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dg_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(dg):
+    names = declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(dg.library, n), f"libdg.so does not export {n}"
+    out = subprocess.run(["nm", "-D", "--defined-only", dg.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    for n in names:
+        assert re.search(rf"\bT {n}\b", out), f"{n} is not a defined text symbol"
+
+
+def test_config_struct_layout_matches_header(dg, tmp_path):
+    fields = [f for f, _ in dg.DgConfig._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "dg.h"\nint main(void){\n'
+                   '  printf("%zu\\n", sizeof(dg_config));\n' +
+                   "".join(f'  printf("%zu\\n", offsetof(dg_config, {f}));\n' for f in fields) +
+                   "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    vals = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True,
+                                           check=True).stdout.split()]
+    assert vals[0] == ctypes.sizeof(dg.DgConfig)
+    for f, off in zip(fields, vals[1:]):
+        assert getattr(dg.DgConfig, f).offset == off, f
+
+
+def test_invalid_configs_rejected_before_device_use(dg):
+    import synth
+    base = synth.config("tiny")
+    bad = [dict(d_model=100), dict(head_dim=96), dict(n_q_heads=3), dict(top_k=9),
+           dict(canvas_len=300), dict(mask_id=1024), dict(n_shared=2), dict(d_ff=100)]
+    for b in bad:
+        cfg = dg.config_from_dict(dict(base, **b))
+        out = ctypes.c_void_p()
+        rc = dg.raw_call("dg_create", ctypes.byref(cfg), None, ctypes.byref(out))
+        assert rc == dg.DG_ERR_INVALID_ARG, b
+        assert out.value is None
+        assert dg.dg_last_error(None) != ""
+
+
+def test_null_arguments_and_no_device(dg):
+    import synth
+    cfg = dg.config_from_dict(synth.config("tiny"))
+    assert dg.raw_call("dg_create", None, None, None) == dg.DG_ERR_INVALID_ARG
+    out = ctypes.c_void_p()
+    rc = dg.raw_call("dg_create", ctypes.byref(cfg), None, ctypes.byref(out))
+    import torch
+    if not torch.cuda.is_available():
+        assert rc == dg.DG_ERR_CUDA and out.value is None
+        assert "device" in dg.dg_last_error(None)
+    else:
+        assert rc == dg.DG_OK
+        dg.dg_destroy(out.value)
+    for name, args in [("dg_init_weights", (None, 0)), ("dg_sync", (None,)),
+                       ("dg_canvas_step", (None, None, 1, 1, None, None)),
+                       ("dg_denoise_block", (None, None, 1, 1)),
+                       ("dg_layer_forward", (None, 0, None, None, 1)),
+                       ("dg_set_prompt_kv", (None, 0, None, None, 1, 1)),
+                       ("dg_router_topk", (None, None, 1, None, None, None, None)),
+                       ("dg_commit", (None, None, None, 1, 1, None, None))]:
+        assert dg.raw_call(name, *args) == dg.DG_ERR_INVALID_ARG, name
+    dg.dg_destroy(None)
+    assert dg.dg_device_bytes(None) == 0

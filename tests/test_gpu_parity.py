@@ -1,0 +1,336 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Tolerances: bf16 layer outputs within relative L2 1e-2; router indices,
+permutations and commit decisions bit-exact when both sides see identical
+scores (ties toward the lower index).  Intermediate stages are checked with
+teacher forcing: the oracle step is fed the device's own input to that step,
+so each kernel is judged alone.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import model as om
+from oracle import rng as orng
+from tests.gpu_helpers import Ctx, bf16_bits, oracle_weight_bits, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+LAYER_TOL = 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    from canvas_denoising_step_b200.build import build
+    build()
+    torch.cuda.set_device(0)
+
+
+def gpu_cfg(name, **kw):
+    return synth.config(name, bf16_weights=True, **kw)
+
+
+# ----------------------------------------------------------------------------- weights
+
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_device_weights_bit_exact_with_oracle_generator(name):
+    cfg = gpu_cfg(name)
+    c = Ctx(cfg, with_prompt=False)
+    try:
+        d, F, E, dh = cfg["d_model"], cfg["d_ff"], cfg["n_experts"], cfg["head_dim"]
+        Hq, Hkv = cfg["n_q_heads"], cfg["n_kv_heads"]
+        lt = orng.layer_tid
+        assert np.array_equal(c.fetch_bits("embed"),
+                              oracle_weight_bits(cfg, orng.EMBED_TID, (cfg["vocab"], d)).ravel())
+        for l in range(cfg["n_layers"]):
+            qkv = np.concatenate([oracle_weight_bits(cfg, lt(l, "wq"), (Hq * dh, d)),
+                                  oracle_weight_bits(cfg, lt(l, "wk"), (Hkv * dh, d)),
+                                  oracle_weight_bits(cfg, lt(l, "wv"), (Hkv * dh, d))])
+            assert np.array_equal(c.fetch_bits(f"wqkv:{l}"), qkv.ravel())
+            assert np.array_equal(c.fetch_bits(f"wo:{l}"),
+                                  oracle_weight_bits(cfg, lt(l, "wo"), (d, Hq * dh)).ravel())
+            assert np.array_equal(c.fetch_bits(f"wr:{l}"),
+                                  oracle_weight_bits(cfg, lt(l, "wr"), (E, d)).ravel())
+            gu = c.fetch_bits(f"wgu:{l}").reshape(E + 1, 2 * F, d)
+            dn = c.fetch_bits(f"wd:{l}").reshape(E + 1, d, F)
+            assert np.array_equal(gu[0, 0::2], oracle_weight_bits(cfg, lt(l, "sg"), (F, d)))
+            assert np.array_equal(gu[0, 1::2], oracle_weight_bits(cfg, lt(l, "su"), (F, d)))
+            assert np.array_equal(dn[0], oracle_weight_bits(cfg, lt(l, "sd"), (d, F)))
+            for e in (0, 1, E - 1):
+                assert np.array_equal(gu[e + 1, 0::2], oracle_weight_bits(cfg, lt(l, "wg"), (F, d),
+                                                                          start=e * F * d))
+                assert np.array_equal(gu[e + 1, 1::2], oracle_weight_bits(cfg, lt(l, "wu"), (F, d),
+                                                                          start=e * F * d))
+                assert np.array_equal(dn[e + 1], oracle_weight_bits(cfg, lt(l, "wd"), (d, F),
+                                                                    start=e * d * F))
+    finally:
+        c.close()
+
+
+# ----------------------------------------------------------------------------- router / commit hooks
+
+def test_router_hook_bit_exact():
+    cfg = gpu_cfg("ragged")
+    c = Ctx(cfg, with_prompt=False)
+    try:
+        T, E, k = c.T, cfg["n_experts"], cfg["top_k"]
+        g = np.random.default_rng(7)
+        logits = g.standard_normal((T, E)).astype(np.float32)
+        logits[0, [3, 5, 9, 11, 12]] = 2.5            # five-way tie for the top slots
+        logits[1, :] = 0.25                            # all equal
+        logits[2, [0, E - 1]] = 9.0
+        dl = torch.from_numpy(logits).cuda()
+        idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+        w = torch.empty(T, k, device="cuda")
+        off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+        perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+        c.dg.dg_router_topk(c.ctx, dl.data_ptr(), T, idx.data_ptr(), w.data_ptr(),
+                            off.data_ptr(), perm.data_ptr())
+        c.dg.dg_sync(c.ctx)
+        ref_idx, ref_w = om.router_topk(logits, k)
+        ref_off, ref_perm = om.router_permutation(ref_idx, E)
+        assert np.array_equal(idx.cpu().numpy(), ref_idx)
+        assert np.array_equal(off.cpu().numpy(), ref_off)
+        assert np.array_equal(perm.cpu().numpy(), ref_perm)
+        assert np.allclose(w.cpu().numpy(), ref_w, rtol=2e-6, atol=1e-7)
+    finally:
+        c.close()
+
+
+def test_commit_hook_bit_exact():
+    cfg = gpu_cfg("ragged")
+    c = Ctx(cfg, with_prompt=False)
+    try:
+        B, Tc, mask = c.B, c.Tc, cfg["mask_id"]
+        g = np.random.default_rng(3)
+        canvas = np.where(g.uniform(size=(B, Tc)) < 0.3, 17, mask).astype(np.int32)
+        conf = g.uniform(size=(B, Tc)).astype(np.float32)
+        conf[0, 5:15] = 0.75                           # ties among masked slots
+        tok = g.integers(1, cfg["vocab"], size=(B, Tc)).astype(np.int32)
+        for steps_left in (1, 2, 3, 7):
+            dcan = torch.from_numpy(canvas).cuda()
+            com = torch.empty(B, Tc, dtype=torch.uint8, device="cuda")
+            c.dg.dg_commit(c.ctx, torch.from_numpy(conf).cuda().data_ptr(), dcan.data_ptr(), B,
+                           steps_left, torch.from_numpy(tok).cuda().data_ptr(), com.data_ptr())
+            c.dg.dg_sync(c.ctx)
+            ref_can, ref_com = om.commit(canvas, conf, tok, steps_left, mask)
+            assert np.array_equal(dcan.cpu().numpy(), ref_can), steps_left
+            assert np.array_equal(com.cpu().numpy().astype(bool), ref_com), steps_left
+    finally:
+        c.close()
+
+
+# ----------------------------------------------------------------------------- one layer
+
+def _layer_check(name, layer, **kw):
+    cfg = gpu_cfg(name, **kw)
+    c = Ctx(cfg)
+    try:
+        oc, B, Tc, T, P = c.oc, c.B, c.Tc, c.T, c.P
+        d, dh, Hq, Hkv = cfg["d_model"], cfg["head_dim"], cfg["n_q_heads"], cfg["n_kv_heads"]
+        E, k = cfg["n_experts"], cfg["top_k"]
+        x_in = synth.hidden_states(cfg)
+        xd = x_in.cuda()
+        out = torch.empty_like(xd)
+        c.dg.dg_layer_forward(c.ctx, layer, xd.data_ptr(), out.data_ptr(), T)
+        c.dg.dg_sync(c.ctx)
+        got = out.float().cpu().numpy().reshape(B, Tc, d)
+        q = c.fetch("q", torch.bfloat16, (B, Hq, Tc, dh))
+        kc = c.fetch("kc", torch.bfloat16, (B, Hkv, Tc, dh))
+        vc = c.fetch("vc", torch.bfloat16, (B, Hkv, Tc, dh))
+        attn_o = c.fetch("attn_o", torch.bfloat16, (B, Tc, Hq, dh))
+        x2 = c.fetch("x2", torch.bfloat16, (T, d))
+        logits = c.fetch("router_logits", torch.float32, (T, E))
+        idx = c.fetch("idx", torch.int32, (T, k))
+        w = c.fetch("w", torch.float32, (T, k))
+        offs = c.fetch("offsets", torch.int32, (E + 1,))
+        perm = c.fetch("perm", torch.int32, (T * k,))
+
+        W = om.layer_weights(oc, layer)
+        h = x_in.float().numpy().astype(np.float64).reshape(B, Tc, d)
+        tr = {}
+        ref = om.layer_forward(oc, W, h, [kv[0] for kv in c.kv_host][layer],
+                               [kv[1] for kv in c.kv_host][layer], trace=tr)
+        report = {}
+        # projections + RoPE
+        n_rot = om.rope_pairs_rotated(oc, layer)
+        pos = P + np.arange(Tc)
+        for b in range(B):
+            qr = om.rope_rotate(tr["q"][b], pos, oc.rope_theta, n_rot)      # [Tc, Hq, dh]
+            kr = om.rope_rotate(tr["k"][b], pos, oc.rope_theta, n_rot)
+            report.setdefault("q", []).append(rel_l2(q[b].transpose(1, 0, 2), qr))
+            report.setdefault("k", []).append(rel_l2(kc[b].transpose(1, 0, 2), kr))
+            report.setdefault("v", []).append(rel_l2(vc[b].transpose(1, 0, 2), tr["v"][b]))
+        # attention, teacher-forced on the device's q / k / v
+        n_vis = P if om.is_global_layer(oc, layer) else min(oc.window, P)
+        kp, vp = c.kv_host[layer]
+        for b in range(B):
+            o_ref = om.attention(q[b].transpose(1, 0, 2), kc[b].transpose(1, 0, 2),
+                                 vc[b].transpose(1, 0, 2), kp[b], vp[b], n_vis)
+            report.setdefault("attn", []).append(rel_l2(attn_o[b], o_ref))
+        # output projection + norms, teacher-forced on the device's attention output
+        attn = attn_o.reshape(T, Hq * dh).astype(np.float64) @ W.get("wo").T
+        h1 = h.reshape(T, d) + om.rmsnorm(attn, 1.0, oc.rms_eps)
+        x2_ref = om.rmsnorm(h1, 1.0, oc.rms_eps)
+        report["x2"] = rel_l2(x2, x2_ref)
+        # router logits on the device's x2; selection / grouping on the device's logits
+        report["logits"] = rel_l2(logits, x2.astype(np.float64) @ W.get("wr").T)
+        ridx, rw = om.router_topk(logits, k)
+        roff, rperm = om.router_permutation(idx, E)
+        assert np.array_equal(idx, ridx), "router selection differs on identical logits"
+        assert np.allclose(w, rw, rtol=1e-5, atol=1e-7)
+        assert np.array_equal(offs, roff) and np.array_equal(perm, rperm)
+        # MoE on the device's x2 and selection
+        y, _, _, _ = om.moe_ffn(oc, W, x2.astype(np.float64), forced_idx=idx)
+        report["moe_out"] = rel_l2(got.reshape(T, d), h1 + y)
+        # whole layer, oracle end to end
+        flips = int((tr["idx"] != idx).any(axis=1).sum())
+        report["layer"] = rel_l2(got, ref)
+        report["router_rows_flipped"] = flips
+        print(name, layer, report)
+        for key in ("q", "k", "v", "attn"):
+            assert max(report[key]) < LAYER_TOL, (key, report)
+        for key in ("x2", "moe_out"):
+            assert report[key] < LAYER_TOL, (key, report)
+        assert report["logits"] < 1e-4, report
+        if flips == 0:
+            assert report["layer"] < LAYER_TOL, report
+        else:
+            assert report["layer"] < 5 * LAYER_TOL, report
+        return report
+    finally:
+        c.close()
+
+
+@pytest.mark.parametrize("name,layer", [("tiny", 0), ("tiny", 1), ("ragged", 0), ("ragged", 1)])
+def test_layer_parity(name, layer):
+    _layer_check(name, layer)
+
+
+def test_layer_parity_rope_off_and_no_shared():
+    _layer_check("ragged", 1, rope_enabled=False, n_shared=0)
+
+
+# ----------------------------------------------------------------------------- full step
+
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_canvas_step_head_and_commit(name):
+    cfg = gpu_cfg(name)
+    c = Ctx(cfg)
+    try:
+        oc, B, Tc, T = c.oc, c.B, c.Tc, c.T
+        canvas0 = synth.initial_canvas(cfg).numpy()
+        canvas = torch.from_numpy(canvas0).cuda()
+        conf = torch.empty(B, Tc, device="cuda")
+        com = torch.empty(B, Tc, dtype=torch.uint8, device="cuda")
+        S = cfg["steps"]
+        c.dg.dg_canvas_step(c.ctx, canvas.data_ptr(), B, S, conf.data_ptr(), com.data_ptr())
+        c.dg.dg_sync(c.ctx)
+        hn = c.fetch("hn", torch.bfloat16, (T, cfg["d_model"]))
+        tok = c.fetch("tok", torch.int32, (T,))
+        conf_np = conf.cpu().numpy()
+        # vocab head on the device's final hidden states
+        rconf, rtok, rm, _ = om.head_reduce(oc, hn.astype(np.float64))
+        assert np.allclose(conf_np.ravel(), rconf, rtol=1e-3)
+        assert np.array_equal(tok, rtok)
+        # commit on the device's confidences: bit-exact
+        ref_can, ref_com = om.commit(canvas0, conf_np, tok.reshape(B, Tc), S, cfg["mask_id"])
+        assert np.array_equal(canvas.cpu().numpy(), ref_can)
+        assert np.array_equal(com.cpu().numpy().astype(bool), ref_com)
+        # whole pass against the oracle end to end
+        o_can, o_conf, o_tok, _ = om.canvas_step(oc, canvas0, [kv[0] for kv in c.kv_host],
+                                                 [kv[1] for kv in c.kv_host], S)
+        err = np.abs(np.log(conf_np) - np.log(o_conf)).max()
+        print(name, "end-to-end max |log conf diff|", err,
+              "argmax agreement", float((o_tok == tok.reshape(B, Tc)).mean()))
+        assert err < 5e-2
+    finally:
+        c.close()
+
+
+def test_denoise_block_invariants_and_resume():
+    cfg = gpu_cfg("ragged")
+    c = Ctx(cfg)
+    try:
+        B, Tc, S, mask = c.B, c.Tc, cfg["steps"], cfg["mask_id"]
+        canvas0 = synth.initial_canvas(cfg).cuda()
+        # step by step
+        cur = canvas0.clone()
+        masked = [int((cur == mask).sum())]
+        prev = cur.cpu().numpy()
+        for s in range(S):
+            com = torch.empty(B, Tc, dtype=torch.uint8, device="cuda")
+            c.dg.dg_canvas_step(c.ctx, cur.data_ptr(), B, S - s, None, com.data_ptr())
+            c.dg.dg_sync(c.ctx)
+            now = cur.cpu().numpy()
+            keep = prev != mask
+            assert np.array_equal(now[keep], prev[keep]), "a committed slot changed"
+            r_before = (prev == mask).sum(axis=1)
+            k_expect = -(-r_before // (S - s))
+            assert np.array_equal(com.cpu().numpy().sum(axis=1), k_expect)
+            masked.append(int((now == mask).sum()))
+            prev = now
+        assert masked[-1] == 0
+        assert all(a >= b for a, b in zip(masked, masked[1:]))
+        # one call for the whole block gives the same tokens (deterministic path)
+        blk = canvas0.clone()
+        c.dg.dg_denoise_block(c.ctx, blk.data_ptr(), B, S)
+        assert np.array_equal(blk.cpu().numpy(), prev)
+        # resume: one step, then the remaining S-1 in a block
+        r = canvas0.clone()
+        c.dg.dg_canvas_step(c.ctx, r.data_ptr(), B, S, None, None)
+        c.dg.dg_denoise_block(c.ctx, r.data_ptr(), B, S - 1)
+        assert np.array_equal(r.cpu().numpy(), prev)
+    finally:
+        c.close()
+
+
+def test_host_buffer_step_matches_device_step():
+    cfg = gpu_cfg("tiny")
+    c = Ctx(cfg)
+    try:
+        B, Tc = c.B, c.Tc
+        a = synth.initial_canvas(cfg).cuda()
+        conf_d = torch.empty(B, Tc, device="cuda")
+        c.dg.dg_canvas_step(c.ctx, a.data_ptr(), B, 2, conf_d.data_ptr(), None)
+        c.dg.dg_sync(c.ctx)
+        h = synth.initial_canvas(cfg).pin_memory()
+        conf_h = torch.empty(B, Tc).pin_memory()
+        com_h = torch.empty(B, Tc, dtype=torch.uint8).pin_memory()
+        c.dg.dg_canvas_step_host(c.ctx, h.data_ptr(), B, 2, conf_h.data_ptr(), com_h.data_ptr())
+        assert np.array_equal(h.numpy(), a.cpu().numpy())
+        assert np.array_equal(conf_h.numpy(), conf_d.cpu().numpy())
+        assert int(com_h.sum()) == 8
+    finally:
+        c.close()
+
+
+def test_bad_state_errors():
+    import canvas_denoising_step_b200 as dg
+    cfg = gpu_cfg("tiny")
+    c = Ctx(cfg, with_prompt=False)
+    try:
+        canvas = synth.initial_canvas(cfg).cuda()
+        with pytest.raises(dg.DgError) as e:
+            dg.dg_canvas_step(c.ctx, canvas.data_ptr(), 1, 1)
+        assert e.value.code == dg.DG_ERR_BAD_STATE
+        with pytest.raises(dg.DgError) as e:
+            dg.dg_canvas_step(c.ctx, canvas.data_ptr(), 1, 0)
+        assert e.value.code == dg.DG_ERR_INVALID_ARG
+        with pytest.raises(dg.DgError) as e:
+            dg.dg_set_prompt_kv(c.ctx, 5, canvas.data_ptr(), canvas.data_ptr(), 1, 8)
+        assert e.value.code == dg.DG_ERR_INVALID_ARG
+    finally:
+        c.close()
+
+
+def test_alloc_limit_gives_oom():
+    import canvas_denoising_step_b200 as dg
+    cfg = gpu_cfg("tiny")
+    with pytest.raises(dg.DgError) as e:
+        dg.dg_create(dg.config_from_dict(cfg, alloc_limit_bytes=1 << 20), 0)
+    assert e.value.code == dg.DG_ERR_OOM
