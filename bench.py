@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""Canvas denoising step benchmark: canvas tokens/sec on one B200 at fixed
+denoise steps, and the fraction of the HBM roofline.
+
+Workload ("stack"): the 30-layer synthetic stack (25 local layers with a
+1024-key window over the prompt, 5 global layers), d_model 2816, 16 query / 8
+key-value heads of 256, 128 experts top-8 + 1 shared (width 704), tied vocab
+262144, a 256-slot canvas, a 4096-token prompt K/V per layer, batch 1, 8
+denoising steps per block.  Weights are seeded random (bf16), the prompt K/V
+and canvas synthetic.
+
+A step is one full pass (embedding, 30 blocks, vocab head, commit) through
+the C ABI.  canvas tok/s = batch * 256 tokens finalised per 8 steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torchrun), every rank runs its own replica on its own
+GPU (independent canvases, no collective on the data path; weak scaling); the
+timed region is bracketed by barriers and the reported time is the max over
+ranks.  --impl reference times the CPU oracle as the reference arm.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "stack"
+
+
+def workload_desc(cfg):
+    return (f"{cfg['n_layers']}-layer canvas denoising stack: d_model {cfg['d_model']}, "
+            f"{cfg['n_q_heads']}q/{cfg['n_kv_heads']}kv heads x {cfg['head_dim']}, "
+            f"{cfg['n_experts']} experts top-{cfg['top_k']} + {cfg['n_shared']} shared "
+            f"(width {cfg['d_ff']}), vocab {cfg['vocab']} tied, canvas {cfg['canvas_len']}, "
+            f"prompt K/V {cfg['prompt_len']} per layer (window {cfg['window']} on 5 of 6 layers), "
+            f"batch {cfg['batch']}, {cfg['steps']} steps per block")
+
+
+def config_json(cfg, n_gpus):
+    return {"workload": workload_desc(cfg), "name": WORKLOAD, "batch": cfg["batch"],
+            "canvas_len": cfg["canvas_len"], "prompt_len": cfg["prompt_len"],
+            "steps_per_block": cfg["steps"], "n_layers": cfg["n_layers"],
+            "l2": "inputs larger than L2: ~50 GB of weights streamed from HBM every step",
+            "parallelism": "replicas" if n_gpus > 1 else "single"}
+
+
+# ----------------------------------------------------------------------------- algorithmic bytes
+
+def bytes_per_step(cfg):
+    """Algorithmic HBM bytes of one pass: every weight once, each layer's visible
+    prompt K/V once, plus the activation tensors the kernels stream."""
+    d, F, E, k = cfg["d_model"], cfg["d_ff"], cfg["n_experts"], cfg["top_k"]
+    dh, Hq, Hkv = cfg["head_dim"], cfg["n_q_heads"], cfg["n_kv_heads"]
+    T = cfg["batch"] * cfg["canvas_len"]
+    P, W, L = cfg["prompt_len"], cfg["window"], cfg["n_layers"]
+    per_layer_w = 2 * ((Hq + 2 * Hkv) * dh * d + d * Hq * dh + E * d + (E + 1) * 3 * F * d)
+    kv = 0
+    for l in range(L):
+        vis = P if (l + 1) % cfg["global_every"] == 0 else min(W, P)
+        kv += 2 * cfg["batch"] * Hkv * vis * dh * 2
+    head = cfg["vocab"] * d * 2
+    return L * per_layer_w + kv + head
+
+
+def gateup_bytes_per_launch(cfg):
+    d, F, E, k = cfg["d_model"], cfg["d_ff"], cfg["n_experts"], cfg["top_k"]
+    T = cfg["batch"] * cfg["canvas_len"]
+    rows = (k + 1) * T
+    return (E + 1) * 2 * F * d * 2 + rows * d * 2 + rows * F * 2
+
+
+def flops_per_step(cfg):
+    d, F, E, k = cfg["d_model"], cfg["d_ff"], cfg["n_experts"], cfg["top_k"]
+    dh, Hq, Hkv = cfg["head_dim"], cfg["n_q_heads"], cfg["n_kv_heads"]
+    T = cfg["batch"] * cfg["canvas_len"]
+    P, W, L, Tc = cfg["prompt_len"], cfg["window"], cfg["n_layers"], cfg["canvas_len"]
+    f = 0
+    for l in range(L):
+        vis = P if (l + 1) % cfg["global_every"] == 0 else min(W, P)
+        f += 2 * T * d * ((Hq + 2 * Hkv) * dh + Hq * dh + E)
+        f += 4 * cfg["batch"] * Hq * Tc * (vis + Tc) * dh
+        f += 2 * T * (k + 1) * 3 * F * d
+    return f + 2 * T * d * cfg["vocab"]
+
+
+# ----------------------------------------------------------------------------- peaks, clocks, traffic
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_src_sha():
+    h = hashlib.sha256()
+    for f in ("gemm_tc.cu", "dg_common.cuh", "dg_kernels.h"):
+        h.update(open(os.path.join(ROOT, "canvas_denoising_step_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken on the
+    current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    j = json.load(open(p)).get(kernel)
+    if not j or j.get("kernel_src_sha") != kernel_src_sha():
+        return None
+    return j.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_rank):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        self.gpu = ids[local_rank] if local_rank < len(ids) else str(local_rank)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Active" in v and
+                          "Not" not in v})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+
+class _CachedWeights:
+    """Oracle layer weights drawn once up front, so the timing excludes generation."""
+
+    def __init__(self, oc, layer):
+        from oracle import model as om
+        self.W = om.layer_weights(oc, layer)
+        for k in ("wq", "wk", "wv", "wo", "wr", "sg", "su", "sd"):
+            self.W.get(k)
+        self._experts = {e: self.W.expert(e) for e in range(oc.n_experts)}
+        self.W.expert = self._experts.__getitem__
+
+
+def oracle_sample(cfg, layers, vocab_fraction_den, seed_rows=0):
+    """Time the oracle on a bounded sample of one pass: full-size layers `layers`
+    (all 256 canvas rows) and a 1/vocab_fraction_den slice of the vocab head.
+    Returns (seconds per layer list, seconds for the head slice)."""
+    import numpy as np
+    import synth
+    from oracle import model as om
+    oc = om.OracleConfig.from_dict(cfg)
+    B, Tc, d = cfg["batch"], cfg["canvas_len"], cfg["d_model"]
+    h = synth.hidden_states(cfg).float().numpy().astype(np.float64).reshape(B, Tc, d)
+    times = []
+    for l in layers:
+        Wc = _CachedWeights(oc, l)
+        k, v = synth.prompt_kv(cfg, l)
+        kp, vp = k.float().numpy().astype(np.float64), v.float().numpy().astype(np.float64)
+        t0 = time.perf_counter()
+        om.layer_forward(oc, Wc.W, h, kp, vp)
+        times.append(time.perf_counter() - t0)
+    nv = cfg["vocab"] // vocab_fraction_den
+    Eb = om.embedding_block(oc, 0, nv)
+    hn = om.rmsnorm(h.reshape(B * Tc, d), 1.0, oc.rms_eps)
+    t0 = time.perf_counter()
+    lg = hn @ Eb.T
+    om.logit_stats(lg, oc.mask_id)
+    t_head = time.perf_counter() - t0
+    return times, t_head
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg):
+    """Oracle, as it stands, on a bounded sample of the workload: one local and one
+    global layer at full size plus 1/32 of the vocab head; the pass time is
+    extrapolated as 25 local + 5 global layers + 32 head slices."""
+    L, ge = cfg["n_layers"], cfg["global_every"]
+    n_glob = L // ge
+    (t_loc, t_glob), t_head = oracle_sample(cfg, [0, ge - 1], 32)
+    t_step = (L - n_glob) * t_loc + n_glob * t_glob + 32 * t_head
+    value = cfg["batch"] * cfg["canvas_len"] / (cfg["steps"] * t_step)
+    return {"value": value, "unit": "canvas tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"one local and one global full-size layer (256 canvas rows) and 1/32 of "
+                       f"the vocab head, weights pre-drawn; pass time extrapolated as "
+                       f"{L - n_glob} local + {n_glob} global layers + 32 head slices "
+                       f"= {t_step:.1f} s")}
+
+
+# ----------------------------------------------------------------------------- arms
+
+def run_reference(args, cfg, rank, world):
+    if rank != 0:
+        return
+    import numpy as np  # noqa: F401
+    L, ge = cfg["n_layers"], cfg["global_every"]
+    per = []
+    for s in range(args.warmup + args.steps):
+        layer = ge - 1 if s % ge == ge - 1 else 0
+        (t_l,), t_h = oracle_sample(cfg, [layer], L)
+        if s >= args.warmup:
+            per.append(L * (t_l + t_h))
+    t_step = statistics.mean(per)
+    value = cfg["batch"] * cfg["canvas_len"] / (cfg["steps"] * t_step)
+    unit = "canvas tokens/s"
+    line = {"metric": "canvas tokens/sec on 1 B200 (fixed denoise steps)", "value": value,
+            "unit": unit, "impl": "reference", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_json(cfg, world),
+            "cpu_baseline": {"value": value, "unit": unit, "cores": blas_threads(),
+                             "kind": "oracle",
+                             "sample": (f"each step: one full-size oracle layer (local on 5 of 6 "
+                                        f"steps, global on 1) plus 1/{L} of the vocab head, "
+                                        f"weights pre-drawn, times {L}")},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, cfg, rank, world, local_rank):
+    import torch
+    import canvas_denoising_step_b200 as dg
+    import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    B, Tc, S, L = cfg["batch"], cfg["canvas_len"], cfg["steps"], cfg["n_layers"]
+    T = B * Tc
+    with torch.cuda.stream(stream):
+        ctx = dg.dg_create(dg.config_from_dict(cfg), stream.cuda_stream)
+        dg.dg_init_weights(ctx, cfg["seed"])
+        kv = []
+        for l in range(L):
+            k, v = synth.prompt_kv(cfg, l)
+            kd, vd = k.to(dev, non_blocking=False), v.to(dev, non_blocking=False)
+            kv.append((kd, vd))
+            dg.dg_set_prompt_kv(ctx, l, kd.data_ptr(), vd.data_ptr(), B, cfg["prompt_len"])
+        canvas0 = synth.initial_canvas(cfg).to(dev)
+        canvas = canvas0.clone()
+    stream.synchronize()
+
+    def run_steps(n, start=0):
+        for s in range(start, start + n):
+            if s % S == 0:
+                canvas.copy_(canvas0, non_blocking=True)
+            dg.dg_canvas_step(ctx, canvas.data_ptr(), B, S - (s % S))
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    with torch.cuda.stream(stream):
+        run_steps(args.warmup)
+        dg.dg_sync(ctx)
+        launches_per_step = dg.dg_last_launch_count(ctx)
+        barrier()
+        stream.synchronize()
+        clocks = ClockSampler(local_rank)
+        clocks.start()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run_steps(args.steps)
+        e1.record(stream)
+        stream.synchronize()
+        clk = clocks.stop()
+        barrier()
+        ms = e0.elapsed_time(e1)
+        dg.dg_sync(ctx)
+
+        # per-kernel breakdown: a second pass of K steps with event records per launch
+        dg.dg_profile_enable(ctx, 1)
+        run_steps(args.steps)
+        kern = {}
+        i = 0
+        while (name := dg.dg_kernel_name(i)) is not None:
+            tot, cnt = dg.dg_profile_read(ctx, name)
+            if cnt:
+                kern[name] = (tot, cnt)
+            i += 1
+        dg.dg_profile_enable(ctx, 0)
+
+        # end to end through the host-buffer entry point
+        hc = synth.initial_canvas(cfg).pin_memory()
+        hconf = torch.empty(B, Tc).pin_memory()
+        hcom = torch.empty(B, Tc, dtype=torch.uint8).pin_memory()
+        h0 = hc.clone()
+        for s in range(min(args.warmup, S)):
+            dg.dg_canvas_step_host(ctx, hc.data_ptr(), B, S - s, hconf.data_ptr(), hcom.data_ptr())
+        barrier()
+        stream.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for s in range(args.steps):
+            if s % S == 0:
+                hc.copy_(h0)
+            dg.dg_canvas_step_host(ctx, hc.data_ptr(), B, S - (s % S), hconf.data_ptr(),
+                                   hcom.data_ptr())
+        f1.record(stream)
+        stream.synchronize()
+        ms_e2e = f0.elapsed_time(f1)
+        barrier()
+
+    t_max, t_e2e_max = ms, ms_e2e
+    if world > 1:
+        t = torch.tensor([ms, ms_e2e], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        t_max, t_e2e_max = float(t[0]), float(t[1])
+    dg.dg_destroy(ctx)
+    if rank != 0:
+        return
+
+    tokens = world * B * Tc * args.steps / S
+    value = tokens / (t_max / 1e3)
+    peak, peak_kind = load_peaks()
+    gu_ms, gu_n = kern.get("gemm_gateup", (float("nan"), 1))
+    gu_bytes = gateup_bytes_per_launch(cfg)
+    achieved = gu_bytes / (gu_ms / gu_n / 1e3) / 1e9
+    step_bytes = bytes_per_step(cfg)
+    step_ms = t_max / args.steps
+    total_prof = sum(v[0] for v in kern.values())
+    line = {
+        "metric": "canvas tokens/sec on 1 B200 (fixed denoise steps); % of HBM roofline per step",
+        "value": value, "unit": "canvas tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_json(cfg, world),
+        "roofline": {"bound": "hbm", "kernel": "gemm_gateup", "achieved": achieved,
+                     "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": peak_kind, "traffic": load_traffic("gemm_gateup"),
+                     "algorithmic_bytes_per_launch": gu_bytes,
+                     "avg_launch_ms": gu_ms / gu_n},
+        "step_roofline": {"bytes": step_bytes, "flops": flops_per_step(cfg),
+                          "achieved_gbs": step_bytes / (step_ms / 1e3) / 1e9,
+                          "frac_of_hbm": step_bytes / (step_ms / 1e3) / 1e9 / peak,
+                          "roofline_ms": step_bytes / (peak * 1e9) * 1e3},
+        "kernels_ms_per_step": {k: v[0] / args.steps for k, v in
+                                sorted(kern.items(), key=lambda kv: -kv[1][0])},
+        "profiled_ms_per_step": total_prof / args.steps,
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": tokens / (t_e2e_max / 1e3), "unit": "canvas tokens/s",
+                "h2d_bytes_per_step": T * 4, "d2h_bytes_per_step": T * 4 + T * 4 + T},
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=32)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    import synth
+    cfg = synth.config(args.workload)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            run_reference(args, cfg, rank, world)
+        else:
+            run_ours(args, cfg, rank, world, local_rank)
+    finally:
+        if world > 1 and args.impl == "ours":
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -67,6 +67,9 @@ _SIGS = {
     "dg_router_topk": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "dg_commit": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p]),
     "dg_debug_tensor": (c_int, [c_void_p, c_char_p, c_void_p, c_size_t, POINTER(c_size_t)]),
+    "dg_profile_enable": (c_int, [c_void_p, c_int]),
+    "dg_profile_read": (c_int, [c_void_p, c_char_p, POINTER(c_double), POINTER(c_int)]),
+    "dg_kernel_name": (c_char_p, [c_int]),
     "dg_sync": (c_int, [c_void_p]),
     "dg_last_error": (c_char_p, [c_void_p]),
     "dg_device_bytes": (c_size_t, [c_void_p]),
@@ -155,6 +158,23 @@ def dg_debug_tensor(ctx: int, name: str, dst: int | None, nbytes: int) -> int:
     _check(ctx, _lib.dg_debug_tensor(ctx, name.encode(), dst, nbytes, ctypes.byref(need)),
            "dg_debug_tensor")
     return need.value
+
+
+def dg_profile_enable(ctx: int, on: bool) -> None:
+    _check(ctx, _lib.dg_profile_enable(ctx, int(on)), "dg_profile_enable")
+
+
+def dg_profile_read(ctx: int, kernel: str) -> tuple[float, int]:
+    """(total device ms, launches) recorded for one kernel kind."""
+    t, n = c_double(0.0), c_int(0)
+    _check(ctx, _lib.dg_profile_read(ctx, kernel.encode(), ctypes.byref(t), ctypes.byref(n)),
+           "dg_profile_read")
+    return t.value, n.value
+
+
+def dg_kernel_name(i: int) -> str | None:
+    n = _lib.dg_kernel_name(i)
+    return n.decode() if n else None
 
 
 def dg_sync(ctx: int) -> None:

@@ -78,6 +78,10 @@ struct dg_ctx {
   CUtensorMap m_x_b, m_x_a, m_attn_o_b, m_xperm_b, m_H_b;
 
   int last_T = 0, last_B = 0, launches = 0;
+  struct ProfRec { int kind; cudaEvent_t a, b; };
+  bool prof_on = false;
+  std::vector<ProfRec> prof;
+  std::vector<cudaEvent_t> ev_pool;
 };
 
 namespace {
@@ -95,11 +99,42 @@ int fail(dg_ctx* c, int code, const std::string& msg) {
       return fail(ctx, DG_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(e_)); \
   } while (0)
 
-#define DG_LAUNCH(ctx, call)   \
-  do {                         \
-    ++(ctx)->launches;         \
-    DG_CUDA(ctx, call);        \
+#define DG_LAUNCH(ctx, kind, call)          \
+  do {                                      \
+    ++(ctx)->launches;                      \
+    const int pi_ = prof_begin(ctx, kind);  \
+    DG_CUDA(ctx, call);                     \
+    prof_end(ctx, pi_);                     \
   } while (0)
+
+enum KernelKind {
+  K_EMBED, K_ROPE_TABLE, K_GEMM_QKV, K_ROPE, K_ATTN, K_ATTN_MERGE, K_GEMM_O, K_POST_ATTN,
+  K_GEMM_ROUTER, K_ROUTER_TOPK, K_ROUTER_SORT, K_GATHER, K_GEMM_GATEUP, K_GEMM_DOWN, K_COMBINE,
+  K_GEMM_HEAD, K_HEAD_MERGE, K_COMMIT, K_NUM_KINDS
+};
+const char* const kKindNames[K_NUM_KINDS] = {
+  "embed_norm", "rope_table", "gemm_qkv", "qkv_rope", "attention", "attn_merge", "gemm_o",
+  "post_attn", "gemm_router", "router_topk", "router_sort", "moe_gather", "gemm_gateup",
+  "gemm_down", "moe_combine", "gemm_head", "head_merge", "commit"};
+
+// Per-launch CUDA events while profiling is on (events come from a growing pool).
+int prof_begin(dg_ctx* c, int kind) {
+  if (!c->prof_on) return -1;
+  const size_t need = 2 * (c->prof.size() + 1);
+  while (c->ev_pool.size() < need) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return -1;
+    c->ev_pool.push_back(e);
+  }
+  const int i = (int)c->prof.size();
+  c->prof.push_back({kind, c->ev_pool[2 * i], c->ev_pool[2 * i + 1]});
+  cudaEventRecord(c->prof[i].a, c->stream);
+  return i;
+}
+
+void prof_end(dg_ctx* c, int i) {
+  if (i >= 0) cudaEventRecord(c->prof[i].b, c->stream);
+}
 
 bool ctx_alloc(dg_ctx* c, void** p, size_t bytes) {
   *p = nullptr;
@@ -169,8 +204,8 @@ int choose_splits(int base_tiles, int n_kb, int num_sms) {
 }
 
 // Dense swap-AB projection: part[s][n][m] = X[n] . W[m] over split s.
-int run_dense(dg_ctx* c, const CUtensorMap& mA, const CUtensorMap& mB, int M, int N, int K,
-              int* splits_out) {
+int run_dense(dg_ctx* c, int kind, const CUtensorMap& mA, const CUtensorMap& mB, int M, int N,
+              int K, int* splits_out) {
   GemmArgs a;
   memset(&a, 0, sizeof(a));
   a.mode = GEMM_DENSE;
@@ -184,7 +219,7 @@ int run_dense(dg_ctx* c, const CUtensorMap& mA, const CUtensorMap& mB, int M, in
   a.err = c->err_dev;
   gemm_plan_smem(a);
   const int tiles = a.m_slabs * n_chunks * a.k_splits;
-  DG_LAUNCH(c, gemm_tc_launch(mA, mB, a, std::min(tiles, c->num_sms), c->stream));
+  DG_LAUNCH(c, kind, gemm_tc_launch(mA, mB, a, std::min(tiles, c->num_sms), c->stream));
   *splits_out = a.k_splits;
   return DG_OK;
 }
@@ -208,7 +243,8 @@ int run_grouped(dg_ctx* c, int mode, const CUtensorMap& mA, const CUtensorMap& m
   a.err = c->err_dev;
   (void)T;
   gemm_plan_smem(a);
-  DG_LAUNCH(c, gemm_tc_launch(mA, mB, a, c->num_sms, c->stream));
+  DG_LAUNCH(c, mode == GEMM_GATEUP ? K_GEMM_GATEUP : K_GEMM_DOWN,
+            gemm_tc_launch(mA, mB, a, c->num_sms, c->stream));
   return DG_OK;
 }
 
@@ -223,8 +259,8 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
   int splits = 1, rc;
 
   // q/k/v projections, RoPE / p-RoPE on the canvas rows
-  if ((rc = run_dense(c, L.m_qkv, c->m_x_b, c->NQKV, T, d, &splits)) != DG_OK) return rc;
-  DG_LAUNCH(c, launch_qkv_rope(c->part, splits, T, Tc, Hq, Hkv, dh, n_rot_pairs(cf, l), c->rope_cos,
+  if ((rc = run_dense(c, K_GEMM_QKV, L.m_qkv, c->m_x_b, c->NQKV, T, d, &splits)) != DG_OK) return rc;
+  DG_LAUNCH(c, K_ROPE, launch_qkv_rope(c->part, splits, T, Tc, Hq, Hkv, dh, n_rot_pairs(cf, l), c->rope_cos,
                                c->rope_sin, c->q, c->kc, c->vc, c->stream));
 
   // one softmax over the visible prompt keys and all canvas keys, split-KV
@@ -242,27 +278,27 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
   at.n_chunks = (NK + at.chunk_keys - 1) / at.chunk_keys;
   at.part_o = c->attn_po; at.part_ml = c->attn_ml;
   at.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)dh));
-  DG_LAUNCH(c, launch_attention(at, c->stream));
-  DG_LAUNCH(c, launch_attn_merge(at, c->attn_o, c->stream));
+  DG_LAUNCH(c, K_ATTN, launch_attention(at, c->stream));
+  DG_LAUNCH(c, K_ATTN_MERGE, launch_attn_merge(at, c->attn_o, c->stream));
 
   // output projection, post-attention norm + residual, pre-FFN norm
-  if ((rc = run_dense(c, L.m_o, c->m_attn_o_b, d, T, Hq * dh, &splits)) != DG_OK) return rc;
-  DG_LAUNCH(c, launch_post_attn(c->part, splits, T, d, L.ln_post, L.ln_ff, cf.rms_eps, c->h,
+  if ((rc = run_dense(c, K_GEMM_O, L.m_o, c->m_attn_o_b, d, T, Hq * dh, &splits)) != DG_OK) return rc;
+  DG_LAUNCH(c, K_POST_ATTN, launch_post_attn(c->part, splits, T, d, L.ln_post, L.ln_ff, cf.rms_eps, c->h,
                                 c->xperm, c->stream));
 
   // router
-  if ((rc = run_dense(c, L.m_r, c->m_xperm_b, E, T, d, &splits)) != DG_OK) return rc;
-  DG_LAUNCH(c, launch_router_topk(c->part, splits, c->has_bias ? c->router_bias : nullptr, T, E,
+  if ((rc = run_dense(c, K_GEMM_ROUTER, L.m_r, c->m_xperm_b, E, T, d, &splits)) != DG_OK) return rc;
+  DG_LAUNCH(c, K_ROUTER_TOPK, launch_router_topk(c->part, splits, c->has_bias ? c->router_bias : nullptr, T, E,
                                   k, c->router_logits, c->idx, c->w, c->bitmap, c->stream));
-  DG_LAUNCH(c, launch_router_sort(c->idx, c->bitmap, T, E, k, cf.n_shared, kGroupedTile,
+  DG_LAUNCH(c, K_ROUTER_SORT, launch_router_sort(c->idx, c->bitmap, T, E, k, cf.n_shared, kGroupedTile,
                                   c->offsets_r, c->offsets_g, c->chunk_prefix, c->perm, c->inv,
                                   c->err_dev, c->stream));
-  DG_LAUNCH(c, launch_moe_gather(c->xperm, c->perm, T, k, d, c->stream));
+  DG_LAUNCH(c, K_GATHER, launch_moe_gather(c->xperm, c->perm, T, k, d, c->stream));
 
   // experts (group 0 = shared expert on all rows), SiLU-gated, then down + combine
   if ((rc = run_grouped(c, GEMM_GATEUP, L.m_gu, c->m_xperm_b, d, 2 * cf.d_ff, T)) != DG_OK) return rc;
   if ((rc = run_grouped(c, GEMM_DOWN, L.m_d, c->m_H_b, cf.d_ff, d, T)) != DG_OK) return rc;
-  DG_LAUNCH(c, launch_moe_combine(c->Y, c->w, c->inv, T, k, cf.n_shared, d, c->h, w_next,
+  DG_LAUNCH(c, K_COMBINE, launch_moe_combine(c->Y, c->w, c->inv, T, k, cf.n_shared, d, c->h, w_next,
                                   cf.rms_eps, c->x, c->stream));
   return DG_OK;
 }
@@ -284,7 +320,7 @@ int check_prompt_state(dg_ctx* c, int batch) {
 
 int ensure_rope(dg_ctx* c, int P) {
   if (c->rope_P != P) {
-    DG_LAUNCH(c, launch_rope_table(c->rope_cos, c->rope_sin, c->cfg.canvas_len,
+    DG_LAUNCH(c, K_ROPE_TABLE, launch_rope_table(c->rope_cos, c->rope_sin, c->cfg.canvas_len,
                                    c->cfg.head_dim / 2, P, (double)c->cfg.rope_theta, c->stream));
     c->rope_P = P;
   }
@@ -298,7 +334,7 @@ int run_step(dg_ctx* c, int B, int steps_left) {
   int rc;
   c->launches = 0;
   if ((rc = ensure_rope(c, c->layers[0].kv_P)) != DG_OK) return rc;
-  DG_LAUNCH(c, launch_embed_norm(c->canvas_dev, c->embed, nullptr, cf.vocab, T, d,
+  DG_LAUNCH(c, K_EMBED, launch_embed_norm(c->canvas_dev, c->embed, nullptr, cf.vocab, T, d,
                                  c->layers[0].ln_in, cf.rms_eps, c->h, c->x, c->err_dev,
                                  c->stream));
   for (int l = 0; l < cf.n_layers; ++l) {
@@ -317,10 +353,10 @@ int run_step(dg_ctx* c, int B, int steps_left) {
   a.err = c->err_dev;
   gemm_plan_smem(a);
   const int tiles = a.n_vblocks * a.n_tblocks;
-  DG_LAUNCH(c, gemm_tc_launch(c->m_x_a, c->m_embed, a, std::min(tiles, c->num_sms), c->stream));
-  DG_LAUNCH(c, launch_head_merge(c->head_m, c->head_s, c->head_a, a.n_vblocks, T, c->conf,
+  DG_LAUNCH(c, K_GEMM_HEAD, gemm_tc_launch(c->m_x_a, c->m_embed, a, std::min(tiles, c->num_sms), c->stream));
+  DG_LAUNCH(c, K_HEAD_MERGE, launch_head_merge(c->head_m, c->head_s, c->head_a, a.n_vblocks, T, c->conf,
                                  c->tok, c->stream));
-  DG_LAUNCH(c, launch_commit(c->conf, c->tok, c->canvas_dev, c->committed_dev, B, cf.canvas_len,
+  DG_LAUNCH(c, K_COMMIT, launch_commit(c->conf, c->tok, c->canvas_dev, c->committed_dev, B, cf.canvas_len,
                              steps_left, nullptr, cf.mask_id, c->stream));
   c->last_T = T;
   c->last_B = B;
@@ -599,7 +635,7 @@ int dg_layer_forward(dg_ctx* c, int layer, const void* x_in, void* x_out, int n_
   int rc;
   c->launches = 0;
   if ((rc = ensure_rope(c, L.kv_P)) != DG_OK) return rc;
-  DG_LAUNCH(c, launch_embed_norm(nullptr, nullptr, static_cast<const bf16*>(x_in), c->cfg.vocab,
+  DG_LAUNCH(c, K_EMBED, launch_embed_norm(nullptr, nullptr, static_cast<const bf16*>(x_in), c->cfg.vocab,
                                  n_rows, d, L.ln_in, c->cfg.rms_eps, c->h, c->x, c->err_dev,
                                  c->stream));
   if ((rc = run_layer(c, layer, B, nullptr)) != DG_OK) return rc;
@@ -680,6 +716,37 @@ int dg_debug_tensor(dg_ctx* c, const char* name, void* dst, size_t bytes, size_t
   return DG_OK;
 }
 
+int dg_profile_enable(dg_ctx* c, int on) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  DG_CUDA(c, cudaStreamSynchronize(c->stream));
+  c->prof.clear();
+  c->prof_on = on != 0;
+  return DG_OK;
+}
+
+int dg_profile_read(dg_ctx* c, const char* kernel, double* total_ms, int* launches) {
+  if (!c || !kernel || !total_ms || !launches) return DG_ERR_INVALID_ARG;
+  int kind = -1;
+  for (int i = 0; i < K_NUM_KINDS; ++i)
+    if (std::string(kernel) == kKindNames[i]) kind = i;
+  if (kind < 0) return fail(c, DG_ERR_INVALID_ARG, "unknown kernel name");
+  DG_CUDA(c, cudaStreamSynchronize(c->stream));
+  double t = 0.0;
+  int n = 0;
+  for (const auto& r : c->prof) {
+    if (r.kind != kind) continue;
+    float ms = 0.f;
+    DG_CUDA(c, cudaEventElapsedTime(&ms, r.a, r.b));
+    t += ms;
+    ++n;
+  }
+  *total_ms = t;
+  *launches = n;
+  return DG_OK;
+}
+
+const char* dg_kernel_name(int i) { return (i >= 0 && i < K_NUM_KINDS) ? kKindNames[i] : nullptr; }
+
 int dg_sync(dg_ctx* c) {
   if (!c) return DG_ERR_INVALID_ARG;
   DG_CUDA(c, cudaStreamSynchronize(c->stream));
@@ -697,6 +764,7 @@ int dg_last_launch_count(const dg_ctx* c) { return c ? c->launches : 0; }
 void dg_destroy(dg_ctx* c) {
   if (!c) return;
   cudaStreamSynchronize(c->stream);
+  for (cudaEvent_t e : c->ev_pool) cudaEventDestroy(e);
   free_all(c);
   delete c;
 }

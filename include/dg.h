@@ -192,6 +192,23 @@ int dg_commit(dg_ctx* ctx, const float* conf, int32_t* canvas, int batch, int st
 int dg_debug_tensor(dg_ctx* ctx, const char* name, void* dst, size_t bytes,
                     size_t* bytes_needed);
 
+/* Instrumentation: with on != 0, every kernel launched by the following
+ * passes is bracketed by CUDA events recorded on the context's stream (this
+ * adds two event records per launch); on == 0 stops recording.  Either call
+ * synchronises the stream and clears earlier records. */
+int dg_profile_enable(dg_ctx* ctx, int on);
+
+/* Sum of the device durations (ms) and the number of launches recorded for
+ * one kernel since dg_profile_enable(ctx, 1).  Synchronises.  Kernel names
+ * are those returned by dg_kernel_name(0 ..): "embed_norm", "rope_table",
+ * "gemm_qkv", "qkv_rope", "attention", "attn_merge", "gemm_o", "post_attn",
+ * "gemm_router", "router_topk", "router_sort", "moe_gather", "gemm_gateup",
+ * "gemm_down", "moe_combine", "gemm_head", "head_merge", "commit". */
+int dg_profile_read(dg_ctx* ctx, const char* kernel, double* total_ms, int* launches);
+
+/* Name of kernel kind i (0-based), or NULL past the last one. */
+const char* dg_kernel_name(int i);
+
 /* Waits for the context's stream and reports (then clears) the device error
  * word: DG_ERR_TIMEOUT or DG_ERR_DEVICE_FAULT if a kernel raised one. */
 int dg_sync(dg_ctx* ctx);

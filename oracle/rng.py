@@ -100,8 +100,8 @@ def round_to_bf16(x: np.ndarray) -> np.ndarray:
     return b.astype(np.uint32).view(np.float32)
 
 
-def weight_tensor(seed: int, tid: int, shape, std: float, bf16: bool,
-                  start: int = 0, chunk: int = 1 << 22) -> np.ndarray:
+def weight_tensor_numpy(seed: int, tid: int, shape, std: float, bf16: bool,
+                        start: int = 0, chunk: int = 1 << 22) -> np.ndarray:
     """The logical tensor ``tid`` (row-major ``shape``) as float32 values.
 
     ``start`` offsets the element counter, so a slice of a larger logical
@@ -117,4 +117,38 @@ def weight_tensor(seed: int, tid: int, shape, std: float, bf16: bool,
         out[c0:c1] = irwin_hall_normal_f32(splitmix64_outputs(key, start + c0, c1 - c0), std)
     if bf16:
         out = round_to_bf16(out)
+    return out.reshape(shape)
+
+
+_C_GEN = None
+
+
+def _c_generator():
+    """The C restatement of the same generator (oracle/csrc/weightgen.c), or None."""
+    global _C_GEN
+    if _C_GEN is None:
+        import ctypes
+        try:
+            from .build_c import build
+            lib = ctypes.CDLL(build())
+            f = lib.oracle_weight_normal
+            f.restype = None
+            f.argtypes = [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int64, ctypes.c_float,
+                          ctypes.c_int, ctypes.c_void_p]
+            _C_GEN = f
+        except Exception:  # no compiler: the numpy path is used
+            _C_GEN = False
+    return _C_GEN or None
+
+
+def weight_tensor(seed: int, tid: int, shape, std: float, bf16: bool, start: int = 0) -> np.ndarray:
+    """As ``weight_tensor_numpy``; drawn by the C restatement when it is available
+    (the two are tested bit-identical)."""
+    f = _c_generator()
+    if f is None:
+        return weight_tensor_numpy(seed, tid, shape, std, bf16, start)
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.float32)
+    scale = np.float32(std * math.sqrt(3.0) / 65536.0)
+    f(splitmix64_stream_key(seed, tid), start, n, float(scale), int(bf16), out.ctypes.data)
     return out.reshape(shape)

@@ -33,11 +33,15 @@ class Ctx:
             for l in range(cfg["n_layers"]):
                 k, v = synth.prompt_kv(cfg, l)
                 kd, vd = k.cuda(), v.cuda()
-                self.kv_host.append((k.float().numpy().astype(np.float64),
-                                     v.float().numpy().astype(np.float64)))
+                self.kv_host.append((k, v))
                 self.kv_dev.append((kd, vd))
                 dg.dg_set_prompt_kv(self.ctx, l, kd.data_ptr(), vd.data_ptr(), self.B, self.P)
         self.oc = om.OracleConfig.from_dict(cfg)
+
+    def kv_np(self, layer: int):
+        """Prompt K, V of one layer as float64 numpy [B, Hkv, P, dh]."""
+        k, v = self.kv_host[layer]
+        return (k.float().numpy().astype(np.float64), v.float().numpy().astype(np.float64))
 
     def close(self):
         if self.ctx:

@@ -111,11 +111,13 @@ def test_commit_hook_bit_exact():
         conf = g.uniform(size=(B, Tc)).astype(np.float32)
         conf[0, 5:15] = 0.75                           # ties among masked slots
         tok = g.integers(1, cfg["vocab"], size=(B, Tc)).astype(np.int32)
+        dconf = torch.from_numpy(conf).cuda()      # kept alive across the async launch
+        dtok = torch.from_numpy(tok).cuda()
         for steps_left in (1, 2, 3, 7):
             dcan = torch.from_numpy(canvas).cuda()
             com = torch.empty(B, Tc, dtype=torch.uint8, device="cuda")
-            c.dg.dg_commit(c.ctx, torch.from_numpy(conf).cuda().data_ptr(), dcan.data_ptr(), B,
-                           steps_left, torch.from_numpy(tok).cuda().data_ptr(), com.data_ptr())
+            c.dg.dg_commit(c.ctx, dconf.data_ptr(), dcan.data_ptr(), B, steps_left,
+                           dtok.data_ptr(), com.data_ptr())
             c.dg.dg_sync(c.ctx)
             ref_can, ref_com = om.commit(canvas, conf, tok, steps_left, mask)
             assert np.array_equal(dcan.cpu().numpy(), ref_can), steps_left
@@ -153,8 +155,8 @@ def _layer_check(name, layer, **kw):
         W = om.layer_weights(oc, layer)
         h = x_in.float().numpy().astype(np.float64).reshape(B, Tc, d)
         tr = {}
-        ref = om.layer_forward(oc, W, h, [kv[0] for kv in c.kv_host][layer],
-                               [kv[1] for kv in c.kv_host][layer], trace=tr)
+        kp, vp = c.kv_np(layer)
+        ref = om.layer_forward(oc, W, h, kp, vp, trace=tr)
         report = {}
         # projections + RoPE
         n_rot = om.rope_pairs_rotated(oc, layer)
@@ -167,7 +169,6 @@ def _layer_check(name, layer, **kw):
             report.setdefault("v", []).append(rel_l2(vc[b].transpose(1, 0, 2), tr["v"][b]))
         # attention, teacher-forced on the device's q / k / v
         n_vis = P if om.is_global_layer(oc, layer) else min(oc.window, P)
-        kp, vp = c.kv_host[layer]
         for b in range(B):
             o_ref = om.attention(q[b].transpose(1, 0, 2), kc[b].transpose(1, 0, 2),
                                  vc[b].transpose(1, 0, 2), kp[b], vp[b], n_vis)
@@ -242,8 +243,9 @@ def test_canvas_step_head_and_commit(name):
         assert np.array_equal(canvas.cpu().numpy(), ref_can)
         assert np.array_equal(com.cpu().numpy().astype(bool), ref_com)
         # whole pass against the oracle end to end
-        o_can, o_conf, o_tok, _ = om.canvas_step(oc, canvas0, [kv[0] for kv in c.kv_host],
-                                                 [kv[1] for kv in c.kv_host], S)
+        kvs = [c.kv_np(l) for l in range(cfg["n_layers"])]
+        o_can, o_conf, o_tok, _ = om.canvas_step(oc, canvas0, [kv[0] for kv in kvs],
+                                                 [kv[1] for kv in kvs], S)
         err = np.abs(np.log(conf_np) - np.log(o_conf)).max()
         print(name, "end-to-end max |log conf diff|", err,
               "argmax agreement", float((o_tok == tok.reshape(B, Tc)).mean()))

@@ -415,3 +415,11 @@ def test_denoise_block_invariants_and_resume():
     c1, _, _, _ = om.canvas_step(cfg, canvas0, kp, vp, 3, weights=weights)
     c3 = om.denoise_block(cfg, c1, kp, vp, 2, weights=weights)
     assert np.array_equal(c3, final)
+
+
+def test_c_generator_matches_numpy_generator():
+    for tid, shape, start, bf16 in [(1, (37, 64), 0, True), (77, (5, 1000), 12345, False),
+                                    (64 * 3 + 5, (3, 2816), 7 * 704 * 2816, True)]:
+        a = orng.weight_tensor_numpy(0, tid, shape, 0.02, bf16, start=start)
+        b = orng.weight_tensor(0, tid, shape, 0.02, bf16, start=start)
+        assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
