@@ -57,27 +57,32 @@ def config_json(cfg, n_gpus):
 
 # ----------------------------------------------------------------------------- algorithmic bytes
 
-def bytes_per_step(cfg):
-    """Algorithmic HBM bytes of one pass: every weight once, each layer's visible
-    prompt K/V once, plus the activation tensors the kernels stream."""
-    d, F, E, k = cfg["d_model"], cfg["d_ff"], cfg["n_experts"], cfg["top_k"]
+def bytes_per_step(cfg, active_experts=None):
+    """Algorithmic HBM bytes of one pass: every weight the pass needs once (the
+    dense projections, the router, the shared expert and the routed experts
+    that receive rows -- `active_experts` per layer on average, all of them when
+    None), each layer's visible prompt K/V once, and the tied embedding once."""
+    d, F, E = cfg["d_model"], cfg["d_ff"], cfg["n_experts"]
     dh, Hq, Hkv = cfg["head_dim"], cfg["n_q_heads"], cfg["n_kv_heads"]
-    T = cfg["batch"] * cfg["canvas_len"]
     P, W, L = cfg["prompt_len"], cfg["window"], cfg["n_layers"]
-    per_layer_w = 2 * ((Hq + 2 * Hkv) * dh * d + d * Hq * dh + E * d + (E + 1) * 3 * F * d)
+    act = E if active_experts is None else active_experts
+    dense = 2 * ((Hq + 2 * Hkv) * dh * d + d * Hq * dh + E * d)
+    experts = 2 * (act + cfg["n_shared"]) * 3 * F * d
     kv = 0
     for l in range(L):
         vis = P if (l + 1) % cfg["global_every"] == 0 else min(W, P)
         kv += 2 * cfg["batch"] * Hkv * vis * dh * 2
     head = cfg["vocab"] * d * 2
-    return L * per_layer_w + kv + head
+    return L * (dense + experts) + kv + head
 
 
-def gateup_bytes_per_launch(cfg):
+def gateup_bytes_per_launch(cfg, active_experts=None):
+    """Weights of the groups that receive rows, the gathered rows read, H written."""
     d, F, E, k = cfg["d_model"], cfg["d_ff"], cfg["n_experts"], cfg["top_k"]
+    act = E if active_experts is None else active_experts
     T = cfg["batch"] * cfg["canvas_len"]
     rows = (k + 1) * T
-    return (E + 1) * 2 * F * d * 2 + rows * d * 2 + rows * F * 2
+    return (act + cfg["n_shared"]) * 2 * F * d * 2 + rows * d * 2 + rows * F * 2
 
 
 def flops_per_step(cfg):
@@ -325,6 +330,9 @@ def run_ours(args, cfg, rank, world, local_rank):
                 kern[name] = (tot, cnt)
             i += 1
         dg.dg_profile_enable(ctx, 0)
+        act = torch.empty(L, dtype=torch.int32, device=dev)
+        dg.dg_debug_tensor(ctx, "expert_active", act.data_ptr(), 4 * L)
+        active_avg = float(act.sum().item()) / (args.steps * L)
 
         # end to end through the host-buffer entry point
         hc = synth.initial_canvas(cfg).pin_memory()
@@ -360,9 +368,9 @@ def run_ours(args, cfg, rank, world, local_rank):
     value = tokens / (t_max / 1e3)
     peak, peak_kind = load_peaks()
     gu_ms, gu_n = kern.get("gemm_gateup", (float("nan"), 1))
-    gu_bytes = gateup_bytes_per_launch(cfg)
+    gu_bytes = gateup_bytes_per_launch(cfg, active_avg)
     achieved = gu_bytes / (gu_ms / gu_n / 1e3) / 1e9
-    step_bytes = bytes_per_step(cfg)
+    step_bytes = bytes_per_step(cfg, active_avg)
     step_ms = t_max / args.steps
     total_prof = sum(v[0] for v in kern.values())
     line = {
@@ -377,6 +385,8 @@ def run_ours(args, cfg, rank, world, local_rank):
                      "algorithmic_bytes_per_launch": gu_bytes,
                      "avg_launch_ms": gu_ms / gu_n},
         "step_roofline": {"bytes": step_bytes, "flops": flops_per_step(cfg),
+                          "active_experts_per_layer": active_avg,
+                          "bytes_if_all_experts": bytes_per_step(cfg),
                           "achieved_gbs": step_bytes / (step_ms / 1e3) / 1e9,
                           "frac_of_hbm": step_bytes / (step_ms / 1e3) / 1e9 / peak,
                           "roofline_ms": step_bytes / (peak * 1e9) * 1e3},
@@ -393,6 +403,55 @@ def run_ours(args, cfg, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_layer_case(args, cfg):
+    """One decoder block (dg_layer_forward) on N(0,1) hidden states -- the
+    single-layer workload -- timed with CUDA events, with the per-kernel table.
+    Not the headline line; used for kernel studies and focused ncu captures."""
+    import torch
+    import canvas_denoising_step_b200 as dg
+    import synth
+
+    torch.cuda.set_device(0)
+    stream = torch.cuda.Stream()
+    B, Tc, layer = cfg["batch"], cfg["canvas_len"], args.layer
+    T = B * Tc
+    with torch.cuda.stream(stream):
+        ctx = dg.dg_create(dg.config_from_dict(cfg), stream.cuda_stream)
+        dg.dg_init_weights(ctx, cfg["seed"])
+        k, v = synth.prompt_kv(cfg, layer)
+        kd, vd = k.cuda(), v.cuda()
+        dg.dg_set_prompt_kv(ctx, layer, kd.data_ptr(), vd.data_ptr(), B, cfg["prompt_len"])
+        x = synth.hidden_states(cfg).cuda()
+        out = torch.empty_like(x)
+        for _ in range(args.warmup):
+            dg.dg_layer_forward(ctx, layer, x.data_ptr(), out.data_ptr(), T)
+        dg.dg_sync(ctx)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            dg.dg_layer_forward(ctx, layer, x.data_ptr(), out.data_ptr(), T)
+        e1.record(stream)
+        stream.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        dg.dg_profile_enable(ctx, 1)
+        for _ in range(args.steps):
+            dg.dg_layer_forward(ctx, layer, x.data_ptr(), out.data_ptr(), T)
+        kern, i = {}, 0
+        while (name := dg.dg_kernel_name(i)) is not None:
+            tot, cnt = dg.dg_profile_read(ctx, name)
+            if cnt:
+                kern[name] = tot / args.steps
+            i += 1
+        dg.dg_profile_enable(ctx, 0)
+        act = torch.empty(cfg["n_layers"], dtype=torch.int32, device="cuda")
+        dg.dg_debug_tensor(ctx, "expert_active", act.data_ptr(), 4 * cfg["n_layers"])
+        dg.dg_destroy(ctx)
+    print(json.dumps({"case": "layer_forward", "workload": args.workload, "layer": layer,
+                      "ms_per_layer": ms, "expert_active": int(act[layer].item()) // args.steps,
+                      "kernels_ms": dict(sorted(kern.items(), key=lambda kv: -kv[1]))}),
+          flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -401,11 +460,20 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=["step", "layer"], default="step",
+                    help="step: full canvas passes (the headline); layer: dg_layer_forward")
+    ap.add_argument("--layer", type=int, default=0)
+    ap.add_argument("--set", action="append", default=[], metavar="KEY=INT",
+                    help="override an integer workload field (kernel studies only)")
     args = ap.parse_args()
-    if args.warmup < 3:
+    if args.warmup < 3 and args.case == "step":
         ap.error("--warmup must be >= 3")
     import synth
-    cfg = synth.config(args.workload)
+    cfg = synth.config(args.workload, **{kv.split("=")[0]: int(kv.split("=")[1])
+                                         for kv in args.set})
+    if args.case == "layer":
+        run_layer_case(args, cfg)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

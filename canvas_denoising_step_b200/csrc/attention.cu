@@ -6,8 +6,9 @@
 // a merge kernel combines the chunks by log-sum-exp.
 //
 // This version runs QK^T and PV on the warp-level bf16 MMA (m16n8k16) with
-// ldmatrix from 128-byte-XOR-swizzled shared memory, cp.async double
-// buffering of the 64-key K/V blocks, and the online softmax in registers.
+// ldmatrix from 128-byte-XOR-swizzled shared memory, cp.async loads of the
+// 64-key K/V blocks (single-buffered so that two CTAs share an SM and hide
+// each other's loads), and the online softmax in registers.
 #include "dg_kernels.h"
 
 namespace dg {
@@ -63,11 +64,11 @@ __device__ __forceinline__ int swz(int row, int col) {
 }
 
 template <int DH>
-__global__ void __launch_bounds__(128, 1) attn_partial_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(128, 2) attn_partial_kernel(const AttnArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   bf16* Qs = reinterpret_cast<bf16*>(smem_raw);
-  bf16* Ks = Qs + kQRows * DH;         // [2][kKeys][DH]
-  bf16* Vs = Ks + 2 * kKeys * DH;      // [2][kKeys][DH]
+  bf16* Ks = Qs + kQRows * DH;         // [kKeys][DH]
+  bf16* Vs = Ks + kKeys * DH;          // [kKeys][DH]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qt = blockIdx.x, chunk = blockIdx.y;
   const int b = blockIdx.z / a.Hkv, g = blockIdx.z % a.Hkv;
@@ -93,10 +94,10 @@ __global__ void __launch_bounds__(128, 1) attn_partial_kernel(const AttnArgs a) 
     const bf16* src = qbase + (size_t)(valid ? qr : 0) * DH + q * 8;
     cp_async16(smem_u32(Qs + swz<DH>(r, q * 8)), src, valid);
   }
-  auto load_kv = [&](int blk, int buf) {
+  auto load_kv = [&](int blk) {
     const int kb0 = k_begin + blk * kKeys;
-    bf16* kd = Ks + buf * kKeys * DH;
-    bf16* vd = Vs + buf * kKeys * DH;
+    bf16* kd = Ks;
+    bf16* vd = Vs;
     for (int c = tid; c < kKeys * CPR; c += 128) {
       const int j = c / CPR, q = c % CPR;
       const int kk = kb0 + j;
@@ -116,7 +117,7 @@ __global__ void __launch_bounds__(128, 1) attn_partial_kernel(const AttnArgs a) 
   };
 
   const int n_blocks = (k_end > k_begin) ? (k_end - k_begin + kKeys - 1) / kKeys : 0;
-  if (n_blocks > 0) load_kv(0, 0);
+  if (n_blocks > 0) load_kv(0);
   cp_async_commit();
 
   float o[DH / 8][4];
@@ -126,16 +127,14 @@ __global__ void __launch_bounds__(128, 1) attn_partial_kernel(const AttnArgs a) 
   const int gq = lane >> 2, tq = lane & 3;
 
   for (int blk = 0; blk < n_blocks; ++blk) {
-    if (blk + 1 < n_blocks) {
-      load_kv(blk + 1, (blk + 1) & 1);
+    if (blk > 0) {
+      load_kv(blk);
       cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
     }
+    cp_async_wait<0>();
     __syncthreads();
-    const bf16* Kb = Ks + (blk & 1) * kKeys * DH;
-    const bf16* Vb = Vs + (blk & 1) * kKeys * DH;
+    const bf16* Kb = Ks;
+    const bf16* Vb = Vs;
 
     // S = Q K^T for this warp's 16 rows x 64 keys
     float s[8][4];
@@ -252,18 +251,21 @@ __global__ void attn_merge_kernel(const AttnArgs a, bf16* out) {
   const int rows_total = a.B * a.Hq * a.Tc;
   const int R = blockIdx.x * (blockDim.x >> 5) + warp;
   if (R >= rows_total) return;
-  float M = -INFINITY;
-  for (int c = 0; c < a.n_chunks; ++c)
-    M = fmaxf(M, a.part_ml[((size_t)c * rows_total + R) * 2]);
+  // lane c holds chunk c's (m, l); n_chunks <= 32
+  float mc = -INFINITY, lc = 0.f;
+  if (lane < a.n_chunks) {
+    const float2 ml = *reinterpret_cast<const float2*>(a.part_ml + ((size_t)lane * rows_total + R) * 2);
+    mc = ml.x;
+    lc = ml.y;
+  }
+  const float M = warp_max(mc);
+  const float wl = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+  const float L = warp_sum(wl * lc);
   float acc[DH / 32];
 #pragma unroll
   for (int j = 0; j < DH / 32; ++j) acc[j] = 0.f;
-  float L = 0.f;
   for (int c = 0; c < a.n_chunks; ++c) {
-    const float* ml = a.part_ml + ((size_t)c * rows_total + R) * 2;
-    if (ml[0] == -INFINITY) continue;
-    const float wgt = exp2f(ml[0] - M);
-    L += wgt * ml[1];
+    const float wgt = __shfl_sync(0xffffffffu, wl, c);
     const float* po = a.part_o + ((size_t)c * rows_total + R) * DH;
 #pragma unroll
     for (int j = 0; j < DH / 32; ++j) acc[j] += wgt * po[lane + 32 * j];
@@ -279,7 +281,7 @@ __global__ void attn_merge_kernel(const AttnArgs a, bf16* out) {
 
 template <int DH>
 cudaError_t launch_attention_t(const AttnArgs& a, cudaStream_t s) {
-  const size_t smem = (size_t)(kQRows + 4 * kKeys) * DH * sizeof(bf16);
+  const size_t smem = (size_t)(kQRows + 2 * kKeys) * DH * sizeof(bf16);
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(attn_partial_kernel<DH>,

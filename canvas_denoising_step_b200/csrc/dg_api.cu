@@ -71,6 +71,7 @@ struct dg_ctx {
   int32_t* canvas_dev = nullptr;
   uint8_t* committed_dev = nullptr;
   int* err_dev = nullptr;
+  int* expert_active = nullptr;   // [n_layers] cumulative count of experts given rows
   float *rope_cos = nullptr, *rope_sin = nullptr;
   int rope_P = -1;
   float* router_bias = nullptr;
@@ -178,6 +179,7 @@ std::string check_config(const dg_config& c) {
   if (c.n_kv_heads < 1 || c.n_q_heads < 1 || c.n_q_heads % c.n_kv_heads) return "n_q_heads must be a positive multiple of n_kv_heads";
   if (c.n_experts < 1 || c.n_experts > 256) return "n_experts must be in [1, 256]";
   if (c.top_k < 1 || c.top_k > c.n_experts || c.top_k > 32) return "top_k must be in [1, min(n_experts, 32)]";
+  if ((c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim > 16384) return "(n_q_heads + 2 n_kv_heads) * head_dim must be <= 16384";
   if (c.n_shared != 0 && c.n_shared != 1) return "n_shared must be 0 or 1";
   if (c.vocab < 2) return "vocab must be >= 2";
   if (c.canvas_len < 1 || c.canvas_len > 256) return "canvas_len must be in [1, 256]";
@@ -292,7 +294,7 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
                                   k, c->router_logits, c->idx, c->w, c->bitmap, c->stream));
   DG_LAUNCH(c, K_ROUTER_SORT, launch_router_sort(c->idx, c->bitmap, T, E, k, cf.n_shared, kGroupedTile,
                                   c->offsets_r, c->offsets_g, c->chunk_prefix, c->perm, c->inv,
-                                  c->err_dev, c->stream));
+                                  c->err_dev, c->expert_active + l, c->stream));
   DG_LAUNCH(c, K_GATHER, launch_moe_gather(c->xperm, c->perm, T, k, d, c->stream));
 
   // experts (group 0 = shared expert on all rows), SiLU-gated, then down + combine
@@ -463,6 +465,7 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
     ok &= alloc_n(c, &c->canvas_dev, T);
     ok &= alloc_n(c, &c->committed_dev, T);
     ok &= alloc_n(c, &c->err_dev, 4);
+    ok &= alloc_n(c, &c->expert_active, cf.n_layers);
     ok &= alloc_n(c, &c->rope_cos, (size_t)cf.canvas_len * dh / 2);
     ok &= alloc_n(c, &c->rope_sin, (size_t)cf.canvas_len * dh / 2);
     ok &= alloc_n(c, &c->router_bias, E);
@@ -478,6 +481,7 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
   // zero the scratch that kernels accumulate into or read before writing
   cudaMemset(c->bitmap, 0, (size_t)E * ((T + 31) / 32) * 4);
   cudaMemset(c->err_dev, 0, 16);
+  cudaMemset(c->expert_active, 0, sizeof(int) * cf.n_layers);
   cudaMemset(c->xperm, 0, rows_moe * d * 2);
   cudaMemset(c->H, 0, rows_moe * F * 2);
   cudaMemset(c->x, 0, Tp * d * 2);
@@ -654,7 +658,7 @@ int dg_router_topk(dg_ctx* c, const float* logits, int n_rows, int32_t* idx, flo
   const int E = c->cfg.n_experts, k = c->cfg.top_k;
   DG_CUDA(c, launch_router_topk_only(logits, n_rows, E, k, idx, w, c->bitmap, c->stream));
   DG_CUDA(c, launch_router_sort(idx, c->bitmap, n_rows, E, k, 0, kGroupedTile, offsets, nullptr,
-                                nullptr, perm, c->inv, c->err_dev, c->stream));
+                                nullptr, perm, c->inv, c->err_dev, nullptr, c->stream));
   return DG_OK;
 }
 
@@ -692,6 +696,7 @@ int dg_debug_tensor(dg_ctx* c, const char* name, void* dst, size_t bytes, size_t
   else if (s == "tok") { src = c->tok; n = T * 4; }
   else if (s == "conf") { src = c->conf; n = T * 4; }
   else if (s == "embed") { src = c->embed; n = (size_t)cf.vocab * d * 2; }
+  else if (s == "expert_active") { src = c->expert_active; n = (size_t)cf.n_layers * 4; }
   else {
     // weights of one layer: "<name>:<layer>"
     const size_t colon = s.find(':');
@@ -721,6 +726,7 @@ int dg_profile_enable(dg_ctx* c, int on) {
   DG_CUDA(c, cudaStreamSynchronize(c->stream));
   c->prof.clear();
   c->prof_on = on != 0;
+  DG_CUDA(c, cudaMemset(c->expert_active, 0, sizeof(int) * c->cfg.n_layers));
   return DG_OK;
 }
 

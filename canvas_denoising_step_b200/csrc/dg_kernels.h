@@ -110,10 +110,11 @@ cudaError_t launch_router_topk(const float* part, int splits, const float* bias,
 // relative to the routed block; offsets_g / chunk_prefix [E+2] describe the
 // grouped-GEMM groups: group 0 = shared expert rows [0, T), group e+1 =
 // expert e rows [T + offsets_r[e], T + offsets_r[e+1]).  Clears the bitmap.
+// active_out (may be NULL) is incremented by the number of experts with rows.
 cudaError_t launch_router_sort(const int32_t* idx, uint32_t* bitmap, int T, int E, int k,
                                int n_shared, int n_tile, int32_t* offsets_r, int32_t* offsets_g,
                                int32_t* chunk_prefix, int32_t* perm, int32_t* inv, int* err,
-                               cudaStream_t s);
+                               int* active_out, cudaStream_t s);
 // xperm[T + p] = xperm[perm[p] / k] for p < k*T (rows [0, T) hold the normed input).
 cudaError_t launch_moe_gather(bf16* xperm, const int32_t* perm, int T, int k, int d,
                               cudaStream_t s);

@@ -180,51 +180,63 @@ cudaError_t launch_rope_table(float* cos_t, float* sin_t, int Tc, int half, int 
   return cudaGetLastError();
 }
 
-// grid (T, Hq + 2 Hkv); one block per (row, head)
-__global__ void qkv_rope_kernel(const float* part, int splits, int T, int Tc, int Hq, int Hkv,
-                                int dh, int n_rot, const float* cos_t, const float* sin_t, bf16* q,
-                                bf16* kc, bf16* vc) {
-  const int t = blockIdx.x, hh = blockIdx.y;
+// One block per canvas row.  Thread u handles the pairs (head, j) numbered
+// threadIdx.x + 256 * u; split-K partials are summed split by split so that
+// each thread's loads of one split are independent of one another.
+constexpr int kRopeMaxPerThread = 32;   // (Hq + 2 Hkv) * dh / 2 <= 8192
+
+__global__ void __launch_bounds__(256) qkv_rope_kernel(const float* part, int splits, int T,
+                                                       int Tc, int Hq, int Hkv, int dh, int n_rot,
+                                                       const float* cos_t, const float* sin_t,
+                                                       bf16* q, bf16* kc, bf16* vc) {
+  const int t = blockIdx.x;
   const int b = t / Tc, i = t % Tc;
   const int nqkv = (Hq + 2 * Hkv) * dh;
   const int half = dh / 2;
-  bf16* dst;
-  bool rotate;
-  if (hh < Hq) {
-    dst = q + (((size_t)b * Hq + hh) * Tc + i) * dh;
-    rotate = true;
-  } else if (hh < Hq + Hkv) {
-    dst = kc + (((size_t)b * Hkv + (hh - Hq)) * Tc + i) * dh;
-    rotate = true;
-  } else {
-    dst = vc + (((size_t)b * Hkv + (hh - Hq - Hkv)) * Tc + i) * dh;
-    rotate = false;
-  }
-  for (int j = threadIdx.x; j < half; j += blockDim.x) {
-    float x0 = 0.f, x1 = 0.f;
-    for (int s = 0; s < splits; ++s) {
-      const float* src = part + ((size_t)s * T + t) * nqkv + (size_t)hh * dh;
-      x0 += src[j];
-      x1 += src[j + half];
+  const int npairs = nqkv / 2;
+  float x0[kRopeMaxPerThread], x1[kRopeMaxPerThread];
+#pragma unroll
+  for (int u = 0; u < kRopeMaxPerThread; ++u) x0[u] = x1[u] = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float* src = part + ((size_t)s * T + t) * nqkv;
+#pragma unroll
+    for (int u = 0; u < kRopeMaxPerThread; ++u) {
+      const int p = threadIdx.x + 256 * u;
+      if (p < npairs) {
+        const int hh = p / half, j = p % half;
+        x0[u] += src[hh * dh + j];
+        x1[u] += src[hh * dh + j + half];
+      }
     }
+  }
+#pragma unroll
+  for (int u = 0; u < kRopeMaxPerThread; ++u) {
+    const int p = threadIdx.x + 256 * u;
+    if (p >= npairs) continue;
+    const int hh = p / half, j = p % half;
+    bf16* dst;
+    bool rotate = true;
+    if (hh < Hq) dst = q + (((size_t)b * Hq + hh) * Tc + i) * dh;
+    else if (hh < Hq + Hkv) dst = kc + (((size_t)b * Hkv + (hh - Hq)) * Tc + i) * dh;
+    else { dst = vc + (((size_t)b * Hkv + (hh - Hq - Hkv)) * Tc + i) * dh; rotate = false; }
+    float a0 = x0[u], a1 = x1[u];
     if (rotate && j < n_rot) {
       const float c = cos_t[i * half + j], sn = sin_t[i * half + j];
-      const float y0 = x0 * c - x1 * sn;
-      const float y1 = x0 * sn + x1 * c;
-      x0 = y0;
-      x1 = y1;
+      const float y0 = a0 * c - a1 * sn;
+      const float y1 = a0 * sn + a1 * c;
+      a0 = y0;
+      a1 = y1;
     }
-    dst[j] = f_to_bf16(x0);
-    dst[j + half] = f_to_bf16(x1);
+    dst[j] = f_to_bf16(a0);
+    dst[j + half] = f_to_bf16(a1);
   }
 }
 
 cudaError_t launch_qkv_rope(const float* part, int splits, int T, int Tc, int Hq, int Hkv, int dh,
                             int n_rot, const float* cos_t, const float* sin_t, bf16* q, bf16* kc,
                             bf16* vc, cudaStream_t s) {
-  dim3 grid(T, Hq + 2 * Hkv);
-  qkv_rope_kernel<<<grid, 128, 0, s>>>(part, splits, T, Tc, Hq, Hkv, dh, n_rot, cos_t, sin_t, q,
-                                       kc, vc);
+  qkv_rope_kernel<<<T, 256, 0, s>>>(part, splits, T, Tc, Hq, Hkv, dh, n_rot, cos_t, sin_t, q, kc,
+                                    vc);
   return cudaGetLastError();
 }
 
@@ -235,16 +247,19 @@ __global__ void post_attn_kernel(const float* part, int splits, int T, int d, co
   __shared__ float red[32];
   const int t = blockIdx.x;
   float a[kMaxPerThread];
+#pragma unroll
+  for (int i = 0; i < kMaxPerThread; ++i) a[i] = 0.f;
+  for (int s = 0; s < splits; ++s) {       // independent loads within one split
+    const float* src = part + ((size_t)s * T + t) * d;
+#pragma unroll
+    for (int i = 0; i < kMaxPerThread; ++i) {
+      const int c = threadIdx.x + i * blockDim.x;
+      if (c < d) a[i] += src[c];
+    }
+  }
   float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxPerThread; ++i) {
-    const int c = threadIdx.x + i * blockDim.x;
-    float v = 0.f;
-    if (c < d)
-      for (int s = 0; s < splits; ++s) v += part[((size_t)s * T + t) * d + c];
-    a[i] = v;
-    ss += v * v;
-  }
+  for (int i = 0; i < kMaxPerThread; ++i) ss += a[i] * a[i];
   ss = block_sum(ss, red);
   const float r1 = rsqrtf(ss / (float)d + eps);
   float ss2 = 0.f;
@@ -286,12 +301,21 @@ __global__ void router_topk_kernel(const float* part, int splits, const float* b
   const int W = (T + 31) / 32;
   float v[8];
 #pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = 0.f;
+  for (int s = 0; s < splits; ++s) {       // independent loads within one split
+    const float* src = part + ((size_t)s * T + t) * E;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E) v[i] += src[e];
+    }
+  }
+#pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int e = lane + 32 * i;
     float x = -INFINITY;
     if (e < E) {
-      x = 0.f;
-      for (int s = 0; s < splits; ++s) x += part[((size_t)s * T + t) * E + e];
+      x = v[i];
       if (bias) x += bias[e];
       if (logits_out) logits_out[(size_t)t * E + e] = x;
       if (x != x) x = -INFINITY;
@@ -299,8 +323,10 @@ __global__ void router_topk_kernel(const float* part, int splits, const float* b
     v[i] = x;
   }
   unsigned taken = 0;
-  float sel_v[32];
-  int sel_i[32];
+  __shared__ float s_sel_v[8][32];
+  __shared__ int s_sel_i[8][32];
+  float* sel_v = s_sel_v[warp];
+  int* sel_i = s_sel_i[warp];
   for (int j = 0; j < k; ++j) {
     float bv = -INFINITY;
     int bi = 0x7fffffff;
@@ -319,9 +345,12 @@ __global__ void router_topk_kernel(const float* part, int splits, const float* b
       if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
     }
     if (bi >= 0 && bi < E && (bi & 31) == lane) taken |= 1u << (bi >> 5);
-    sel_v[j] = bv;
-    sel_i[j] = bi;
+    if (lane == 0) {
+      sel_v[j] = bv;
+      sel_i[j] = bi;
+    }
   }
+  __syncwarp();
   if (lane == 0) {
     const float mx = sel_v[0];
     float den = 0.f;
@@ -357,7 +386,7 @@ cudaError_t launch_router_topk_only(const float* logits, int T, int E, int k, in
 __global__ void router_sort_kernel(const int32_t* idx, uint32_t* bitmap, int T, int E, int k,
                                    int n_shared, int n_tile, int32_t* offsets_r,
                                    int32_t* offsets_g, int32_t* chunk_prefix, int32_t* perm,
-                                   int32_t* inv, int* err) {
+                                   int32_t* inv, int* err, int* active_out) {
   extern __shared__ int sm[];
   const int W = (T + 31) / 32;
   int* prefix = sm;              // [E*W]
@@ -390,6 +419,11 @@ __global__ void router_sort_kernel(const int32_t* idx, uint32_t* bitmap, int T, 
     }
     off[E] = run;
     if (offsets_r) offsets_r[E] = run;
+    if (active_out) {
+      int active = 0;
+      for (int e = 0; e < E; ++e) active += count[e] > 0;
+      atomicAdd(active_out, active);
+    }
     if (offsets_g) offsets_g[E + 1] = T + run;
     if (run != T * k) raise_error(err, kErrFault);
   }
@@ -410,7 +444,7 @@ __global__ void router_sort_kernel(const int32_t* idx, uint32_t* bitmap, int T, 
 cudaError_t launch_router_sort(const int32_t* idx, uint32_t* bitmap, int T, int E, int k,
                                int n_shared, int n_tile, int32_t* offsets_r, int32_t* offsets_g,
                                int32_t* chunk_prefix, int32_t* perm, int32_t* inv, int* err,
-                               cudaStream_t s) {
+                               int* active_out, cudaStream_t s) {
   const int W = (T + 31) / 32;
   const size_t smem = (size_t)(E * W + E + E + 1) * sizeof(int);
   static bool attr = false;
@@ -421,7 +455,7 @@ cudaError_t launch_router_sort(const int32_t* idx, uint32_t* bitmap, int T, int 
     attr = true;
   }
   router_sort_kernel<<<1, 1024, smem, s>>>(idx, bitmap, T, E, k, n_shared, n_tile, offsets_r,
-                                           offsets_g, chunk_prefix, perm, inv, err);
+                                           offsets_g, chunk_prefix, perm, inv, err, active_out);
   return cudaGetLastError();
 }
 
@@ -445,24 +479,47 @@ __global__ void moe_combine_kernel(const float* Y, const float* w, const int32_t
                                    int k, int n_shared, int d, float* h, const float* w_next,
                                    float eps, bf16* x) {
   __shared__ float red[32];
+  __shared__ int srow[33];
+  __shared__ float sw[33];
   const int t = blockIdx.x;
+  if (threadIdx.x < k) {
+    srow[threadIdx.x] = T + inv[(size_t)t * k + threadIdx.x];
+    sw[threadIdx.x] = w[(size_t)t * k + threadIdx.x];
+  }
+  __syncthreads();
   float v[kMaxPerThread];
+#pragma unroll
+  for (int i = 0; i < kMaxPerThread; ++i) {
+    const int c = threadIdx.x + i * blockDim.x;
+    v[i] = (c < d) ? h[(size_t)t * d + c] : 0.f;
+  }
+  float y[kMaxPerThread];
+#pragma unroll
+  for (int i = 0; i < kMaxPerThread; ++i) y[i] = 0.f;
+  for (int j = 0; j < k; ++j) {            // fixed order j = 0 .. k-1
+    const float* src = Y + (size_t)srow[j] * d;
+    const float wj = sw[j];
+#pragma unroll
+    for (int i = 0; i < kMaxPerThread; ++i) {
+      const int c = threadIdx.x + i * blockDim.x;
+      if (c < d) y[i] += wj * src[c];
+    }
+  }
+  if (n_shared) {
+    const float* src = Y + (size_t)t * d;
+#pragma unroll
+    for (int i = 0; i < kMaxPerThread; ++i) {
+      const int c = threadIdx.x + i * blockDim.x;
+      if (c < d) y[i] += src[c];
+    }
+  }
   float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < kMaxPerThread; ++i) {
     const int c = threadIdx.x + i * blockDim.x;
-    float y = 0.f;
-    if (c < d) {
-      for (int j = 0; j < k; ++j) {
-        const int r = T + inv[(size_t)t * k + j];
-        y += w[(size_t)t * k + j] * Y[(size_t)r * d + c];
-      }
-      if (n_shared) y += Y[(size_t)t * d + c];
-      y += h[(size_t)t * d + c];
-      h[(size_t)t * d + c] = y;
-    }
-    v[i] = y;
-    ss += y * y;
+    v[i] += y[i];
+    if (c < d) h[(size_t)t * d + c] = v[i];
+    ss += v[i] * v[i];
   }
   if (w_next) {
     ss = block_sum(ss, red);
