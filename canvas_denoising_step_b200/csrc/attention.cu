@@ -70,6 +70,8 @@ __global__ void __launch_bounds__(128, 2) attn_partial_kernel(const AttnArgs a) 
   bf16* Ks = Qs + kQRows * DH;         // [kKeys][DH]
   bf16* Vs = Ks + kKeys * DH;          // [kKeys][DH]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  griddep_wait();
+  griddep_launch();
   const int qt = blockIdx.x, chunk = blockIdx.y;
   const int b = blockIdx.z / a.Hkv, g = blockIdx.z % a.Hkv;
   const int group = a.Hq / a.Hkv;
@@ -247,6 +249,8 @@ __global__ void __launch_bounds__(128, 2) attn_partial_kernel(const AttnArgs a) 
 
 template <int DH>
 __global__ void attn_merge_kernel(const AttnArgs a, bf16* out) {
+  griddep_wait();
+  griddep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rows_total = a.B * a.Hq * a.Tc;
   const int R = blockIdx.x * (blockDim.x >> 5) + warp;
@@ -291,8 +295,7 @@ cudaError_t launch_attention_t(const AttnArgs& a, cudaStream_t s) {
   }
   const int group = a.Hq / a.Hkv;
   dim3 grid((group * a.Tc + kQRows - 1) / kQRows, a.n_chunks, a.B * a.Hkv);
-  attn_partial_kernel<DH><<<grid, 128, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(attn_partial_kernel<DH>, grid, dim3(128), smem, s, a);
 }
 
 }  // namespace
@@ -310,12 +313,11 @@ cudaError_t launch_attn_merge(const AttnArgs& a, bf16* o, cudaStream_t s) {
   const int rows = a.B * a.Hq * a.Tc;
   const int grid = (rows + 7) / 8;
   switch (a.dh) {
-    case 64: attn_merge_kernel<64><<<grid, 256, 0, s>>>(a, o); break;
-    case 128: attn_merge_kernel<128><<<grid, 256, 0, s>>>(a, o); break;
-    case 256: attn_merge_kernel<256><<<grid, 256, 0, s>>>(a, o); break;
+    case 64: return launch_k(attn_merge_kernel<64>, dim3(grid), dim3(256), 0, s, a, o);
+    case 128: return launch_k(attn_merge_kernel<128>, dim3(grid), dim3(256), 0, s, a, o);
+    case 256: return launch_k(attn_merge_kernel<256>, dim3(grid), dim3(256), 0, s, a, o);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace dg

@@ -5,6 +5,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <string>
 #include <vector>
 
@@ -60,6 +61,7 @@ struct dg_ctx {
   int32_t* idx = nullptr;
   float* w = nullptr;
   uint32_t* bitmap = nullptr;
+  int* router_counter = nullptr;
   int32_t *offsets_r = nullptr, *offsets_g = nullptr, *chunk_prefix = nullptr;
   int32_t *perm = nullptr, *inv = nullptr;
   bf16* H = nullptr;
@@ -79,6 +81,10 @@ struct dg_ctx {
   CUtensorMap m_x_b, m_x_a, m_attn_o_b, m_xperm_b, m_H_b;
 
   int last_T = 0, last_B = 0, launches = 0;
+  int* steps_dev = nullptr;          // steps_left of the pass being run
+  struct StepGraph { cudaGraphExec_t exec = nullptr; int launches = 0; };
+  std::map<int, StepGraph> graphs;   // captured passes, by batch size
+  std::map<int, bool> warm;
   struct ProfRec { int kind; cudaEvent_t a, b; };
   bool prof_on = false;
   std::vector<ProfRec> prof;
@@ -110,12 +116,12 @@ int fail(dg_ctx* c, int code, const std::string& msg) {
 
 enum KernelKind {
   K_EMBED, K_ROPE_TABLE, K_GEMM_QKV, K_ROPE, K_ATTN, K_ATTN_MERGE, K_GEMM_O, K_POST_ATTN,
-  K_GEMM_ROUTER, K_ROUTER_TOPK, K_ROUTER_SORT, K_GATHER, K_GEMM_GATEUP, K_GEMM_DOWN, K_COMBINE,
+  K_GEMM_ROUTER, K_ROUTER, K_GATHER, K_GEMM_GATEUP, K_GEMM_DOWN, K_COMBINE,
   K_GEMM_HEAD, K_HEAD_MERGE, K_COMMIT, K_NUM_KINDS
 };
 const char* const kKindNames[K_NUM_KINDS] = {
   "embed_norm", "rope_table", "gemm_qkv", "qkv_rope", "attention", "attn_merge", "gemm_o",
-  "post_attn", "gemm_router", "router_topk", "router_sort", "moe_gather", "gemm_gateup",
+  "post_attn", "gemm_router", "router", "moe_gather", "gemm_gateup",
   "gemm_down", "moe_combine", "gemm_head", "head_merge", "commit"};
 
 // Per-launch CUDA events while profiling is on (events come from a growing pool).
@@ -177,7 +183,7 @@ std::string check_config(const dg_config& c) {
   if (c.d_ff < 64 || c.d_ff % 64) return "d_ff must be a positive multiple of 64";
   if (c.head_dim != 64 && c.head_dim != 128 && c.head_dim != 256) return "head_dim must be 64, 128 or 256";
   if (c.n_kv_heads < 1 || c.n_q_heads < 1 || c.n_q_heads % c.n_kv_heads) return "n_q_heads must be a positive multiple of n_kv_heads";
-  if (c.n_experts < 1 || c.n_experts > 256) return "n_experts must be in [1, 256]";
+  if (c.n_experts < 4 || c.n_experts > 256 || c.n_experts % 4) return "n_experts must be a multiple of 4 in [4, 256]";
   if (c.top_k < 1 || c.top_k > c.n_experts || c.top_k > 32) return "top_k must be in [1, min(n_experts, 32)]";
   if ((c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim > 16384) return "(n_q_heads + 2 n_kv_heads) * head_dim must be <= 16384";
   if (c.n_shared != 0 && c.n_shared != 1) return "n_shared must be 0 or 1";
@@ -290,11 +296,18 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
 
   // router
   if ((rc = run_dense(c, K_GEMM_ROUTER, L.m_r, c->m_xperm_b, E, T, d, &splits)) != DG_OK) return rc;
-  DG_LAUNCH(c, K_ROUTER_TOPK, launch_router_topk(c->part, splits, c->has_bias ? c->router_bias : nullptr, T, E,
-                                  k, c->router_logits, c->idx, c->w, c->bitmap, c->stream));
-  DG_LAUNCH(c, K_ROUTER_SORT, launch_router_sort(c->idx, c->bitmap, T, E, k, cf.n_shared, kGroupedTile,
-                                  c->offsets_r, c->offsets_g, c->chunk_prefix, c->perm, c->inv,
-                                  c->err_dev, c->expert_active + l, c->stream));
+  {
+    RouterArgs ra;
+    memset(&ra, 0, sizeof(ra));
+    ra.logits_in = c->part; ra.splits = splits;
+    ra.bias = c->has_bias ? c->router_bias : nullptr;
+    ra.T = T; ra.E = E; ra.k = k; ra.n_shared = cf.n_shared; ra.n_tile = kGroupedTile;
+    ra.logits_out = c->router_logits; ra.idx = c->idx; ra.w = c->w;
+    ra.bitmap = c->bitmap; ra.counter = c->router_counter;
+    ra.offsets_r = c->offsets_r; ra.offsets_g = c->offsets_g; ra.chunk_prefix = c->chunk_prefix;
+    ra.perm = c->perm; ra.inv = c->inv; ra.active_out = c->expert_active + l; ra.err = c->err_dev;
+    DG_LAUNCH(c, K_ROUTER, launch_router(ra, c->stream));
+  }
   DG_LAUNCH(c, K_GATHER, launch_moe_gather(c->xperm, c->perm, T, k, d, c->stream));
 
   // experts (group 0 = shared expert on all rows), SiLU-gated, then down + combine
@@ -329,13 +342,13 @@ int ensure_rope(dg_ctx* c, int P) {
   return DG_OK;
 }
 
-// Full pass on c->canvas_dev (batch B), conf/tok into c->conf / c->tok, commit in place.
-int run_step(dg_ctx* c, int B, int steps_left) {
+// The kernels of one pass on c->canvas_dev (batch B): conf/tok into c->conf /
+// c->tok, commit in place with steps_left read from c->steps_dev.
+int record_step(dg_ctx* c, int B) {
   const dg_config& cf = c->cfg;
   const int T = B * cf.canvas_len, d = cf.d_model;
   int rc;
   c->launches = 0;
-  if ((rc = ensure_rope(c, c->layers[0].kv_P)) != DG_OK) return rc;
   DG_LAUNCH(c, K_EMBED, launch_embed_norm(c->canvas_dev, c->embed, nullptr, cf.vocab, T, d,
                                  c->layers[0].ln_in, cf.rms_eps, c->h, c->x, c->err_dev,
                                  c->stream));
@@ -359,8 +372,56 @@ int run_step(dg_ctx* c, int B, int steps_left) {
   DG_LAUNCH(c, K_HEAD_MERGE, launch_head_merge(c->head_m, c->head_s, c->head_a, a.n_vblocks, T, c->conf,
                                  c->tok, c->stream));
   DG_LAUNCH(c, K_COMMIT, launch_commit(c->conf, c->tok, c->canvas_dev, c->committed_dev, B, cf.canvas_len,
-                             steps_left, nullptr, cf.mask_id, c->stream));
+                             -1, c->steps_dev, cf.mask_id, c->stream));
   c->last_T = T;
+  c->last_B = B;
+  return DG_OK;
+}
+
+void drop_graphs(dg_ctx* c) {
+  for (auto& g : c->graphs) cudaGraphExecDestroy(g.second.exec);
+  c->graphs.clear();
+}
+
+bool graphs_enabled(const dg_ctx* c) {
+  const char* e = std::getenv("DG_NO_GRAPH");
+  const bool off = e && e[0] && e[0] != '0';
+  return !off && !c->prof_on && c->stream != nullptr && c->stream != cudaStreamLegacy &&
+         c->stream != cudaStreamPerThread;
+}
+
+// One pass: the kernels run from a CUDA graph captured on the second pass of a
+// given batch size (the first runs directly and sets kernel attributes).
+int run_step(dg_ctx* c, int B, int steps_left) {
+  int rc;
+  if ((rc = ensure_rope(c, c->layers[0].kv_P)) != DG_OK) return rc;
+  DG_CUDA(c, launch_set_int(c->steps_dev, steps_left, c->stream));
+  if (!graphs_enabled(c)) return record_step(c, B);
+  auto it = c->graphs.find(B);
+  if (it == c->graphs.end()) {
+    if (!c->warm[B]) {
+      c->warm[B] = true;
+      return record_step(c, B);
+    }
+    cudaGraph_t g = nullptr;
+    DG_CUDA(c, cudaStreamBeginCapture(c->stream, cudaStreamCaptureModeThreadLocal));
+    rc = record_step(c, B);
+    const cudaError_t e = cudaStreamEndCapture(c->stream, &g);
+    if (rc != DG_OK) {
+      if (g) cudaGraphDestroy(g);
+      return rc;
+    }
+    if (e != cudaSuccess) return fail(c, DG_ERR_CUDA, std::string("graph capture: ") + cudaGetErrorString(e));
+    dg_ctx::StepGraph sg;
+    const cudaError_t e2 = cudaGraphInstantiate(&sg.exec, g, 0);
+    cudaGraphDestroy(g);
+    if (e2 != cudaSuccess) return fail(c, DG_ERR_CUDA, std::string("graph instantiate: ") + cudaGetErrorString(e2));
+    sg.launches = c->launches;
+    it = c->graphs.emplace(B, sg).first;
+  }
+  DG_CUDA(c, cudaGraphLaunch(it->second.exec, c->stream));
+  c->launches = it->second.launches;
+  c->last_T = B * c->cfg.canvas_len;
   c->last_B = B;
   return DG_OK;
 }
@@ -449,6 +510,8 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
     ok &= alloc_n(c, &c->idx, T * k);
     ok &= alloc_n(c, &c->w, T * k);
     ok &= alloc_n(c, &c->bitmap, (size_t)E * ((T + 31) / 32));
+    ok &= alloc_n(c, &c->router_counter, 4);
+    ok &= alloc_n(c, &c->steps_dev, 4);
     ok &= alloc_n(c, &c->offsets_r, E + 1);
     ok &= alloc_n(c, &c->offsets_g, E + 2);
     ok &= alloc_n(c, &c->chunk_prefix, E + 2);
@@ -480,6 +543,7 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
   }
   // zero the scratch that kernels accumulate into or read before writing
   cudaMemset(c->bitmap, 0, (size_t)E * ((T + 31) / 32) * 4);
+  cudaMemset(c->router_counter, 0, 16);
   cudaMemset(c->err_dev, 0, 16);
   cudaMemset(c->expert_active, 0, sizeof(int) * cf.n_layers);
   cudaMemset(c->xperm, 0, rows_moe * d * 2);
@@ -566,6 +630,7 @@ int dg_set_prompt_kv(dg_ctx* c, int layer, const void* k, const void* v, int bat
   if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15)
     return fail(c, DG_ERR_INVALID_ARG, "prompt K/V must be 16-byte aligned");
   Layer& L = c->layers[layer];
+  if (L.kp != k || L.vp != v || L.kv_batch != batch || L.kv_P != n_prompt) drop_graphs(c);
   L.kp = static_cast<const bf16*>(k);
   L.vp = static_cast<const bf16*>(v);
   L.kv_batch = batch;
@@ -575,6 +640,7 @@ int dg_set_prompt_kv(dg_ctx* c, int layer, const void* k, const void* v, int bat
 
 int dg_set_router_bias(dg_ctx* c, const float* bias) {
   if (!c) return DG_ERR_INVALID_ARG;
+  drop_graphs(c);
   if (!bias) { c->has_bias = false; return DG_OK; }
   DG_CUDA(c, cudaMemcpyAsync(c->router_bias, bias, sizeof(float) * c->cfg.n_experts,
                              cudaMemcpyDefault, c->stream));
@@ -655,10 +721,16 @@ int dg_router_topk(dg_ctx* c, const float* logits, int n_rows, int32_t* idx, flo
   if (!c) return DG_ERR_INVALID_ARG;
   if (!logits || !idx || !w || !offsets || !perm) return fail(c, DG_ERR_INVALID_ARG, "null argument");
   if (n_rows < 1 || n_rows > c->Tmax) return fail(c, DG_ERR_INVALID_ARG, "n_rows out of range");
-  const int E = c->cfg.n_experts, k = c->cfg.top_k;
-  DG_CUDA(c, launch_router_topk_only(logits, n_rows, E, k, idx, w, c->bitmap, c->stream));
-  DG_CUDA(c, launch_router_sort(idx, c->bitmap, n_rows, E, k, 0, kGroupedTile, offsets, nullptr,
-                                nullptr, perm, c->inv, c->err_dev, nullptr, c->stream));
+  if (reinterpret_cast<uintptr_t>(logits) & 15)
+    return fail(c, DG_ERR_INVALID_ARG, "logits must be 16-byte aligned");
+  RouterArgs ra;
+  memset(&ra, 0, sizeof(ra));
+  ra.logits_in = logits; ra.splits = 1;
+  ra.T = n_rows; ra.E = c->cfg.n_experts; ra.k = c->cfg.top_k; ra.n_shared = 0;
+  ra.n_tile = kGroupedTile;
+  ra.idx = idx; ra.w = w; ra.bitmap = c->bitmap; ra.counter = c->router_counter;
+  ra.offsets_r = offsets; ra.perm = perm; ra.inv = c->inv; ra.err = c->err_dev;
+  DG_CUDA(c, launch_router(ra, c->stream));
   return DG_OK;
 }
 
@@ -726,7 +798,7 @@ int dg_profile_enable(dg_ctx* c, int on) {
   DG_CUDA(c, cudaStreamSynchronize(c->stream));
   c->prof.clear();
   c->prof_on = on != 0;
-  DG_CUDA(c, cudaMemset(c->expert_active, 0, sizeof(int) * c->cfg.n_layers));
+  if (on) DG_CUDA(c, cudaMemset(c->expert_active, 0, sizeof(int) * c->cfg.n_layers));
   return DG_OK;
 }
 
@@ -771,6 +843,7 @@ void dg_destroy(dg_ctx* c) {
   if (!c) return;
   cudaStreamSynchronize(c->stream);
   for (cudaEvent_t e : c->ev_pool) cudaEventDestroy(e);
+  drop_graphs(c);
   free_all(c);
   delete c;
 }

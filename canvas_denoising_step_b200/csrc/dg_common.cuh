@@ -246,6 +246,38 @@ __host__ __device__ __forceinline__ uint32_t idesc_bf16_f32(int n, bool a_mn_maj
          | ((uint32_t)(128 >> 4) << 24);  // M / 16
 }
 
+// ----------------------------------------------------------------------------- PDL
+// Kernels are launched with programmatic stream serialization: a kernel may be
+// scheduled while its predecessor on the stream drains.  Every kernel calls
+// griddep_wait() before it reads or writes any global memory that another
+// kernel touches (the wait returns once the predecessor grid has completed
+// and its writes are visible; completion is transitive along the stream),
+// then griddep_launch() to let its own successor be scheduled.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+bool pdl_enabled();  // false when the environment sets DG_NO_PDL
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 __device__ __forceinline__ float bf16_to_f(bf16 x) { return __bfloat162float(x); }
 __device__ __forceinline__ bf16 f_to_bf16(float x) { return __float2bfloat16_rn(x); }
 

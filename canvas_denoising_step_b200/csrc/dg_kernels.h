@@ -62,6 +62,7 @@ struct InitArgs {
 unsigned long long stream_key_host(unsigned long long seed, unsigned long long tid);
 cudaError_t launch_init(const InitArgs& a, cudaStream_t s);
 cudaError_t launch_fill_f32(float* p, long long n, float v, cudaStream_t s);
+cudaError_t launch_set_int(int* p, int v, cudaStream_t s);
 
 // ---------------------------------------------------------------- elementwise / norm
 // h[t] = float(E[canvas[t]]) (or float(x_in[t]) when x_in != NULL);
@@ -102,19 +103,33 @@ cudaError_t launch_attn_merge(const AttnArgs& a, bf16* o, cudaStream_t s);
 cudaError_t launch_post_attn(const float* part, int splits, int T, int d, const float* w_post,
                              const float* w_ff, float eps, float* h, bf16* x2, cudaStream_t s);
 
-// Router: logits = sum partials (+bias); top-k; weights; bitmap of expert membership.
-cudaError_t launch_router_topk(const float* part, int splits, const float* bias, int T, int E,
-                               int k, float* logits_out, int32_t* idx, float* w,
-                               uint32_t* bitmap, cudaStream_t s);
-// Counting sort (single CTA).  Routed offsets_r [E+1] and perm/inv [T*k] are
-// relative to the routed block; offsets_g / chunk_prefix [E+2] describe the
-// grouped-GEMM groups: group 0 = shared expert rows [0, T), group e+1 =
-// expert e rows [T + offsets_r[e], T + offsets_r[e+1]).  Clears the bitmap.
-// active_out (may be NULL) is incremented by the number of experts with rows.
-cudaError_t launch_router_sort(const int32_t* idx, uint32_t* bitmap, int T, int E, int k,
-                               int n_shared, int n_tile, int32_t* offsets_r, int32_t* offsets_g,
-                               int32_t* chunk_prefix, int32_t* perm, int32_t* inv, int* err,
-                               int* active_out, cudaStream_t s);
+// Router (one kernel): logits = sum of split-K partials (+ bias); top-k per row
+// (value desc, index asc); weights = softmax over the chosen logits; then the
+// last block groups the assignments by expert.  Routed offsets_r [E+1] and
+// perm/inv [T*k] are relative to the routed block; offsets_g / chunk_prefix
+// [E+2] describe the grouped-GEMM groups: group 0 = shared expert rows
+// [0, T), group e+1 = expert e rows [T + offsets_r[e], T + offsets_r[e+1]).
+// The bitmap must be zero on entry and is left zero; counter likewise.
+struct RouterArgs {
+  const float* logits_in;  // [splits][T][E] fp32
+  int splits;
+  const float* bias;       // [E] or NULL
+  int T, E, k, n_shared, n_tile;
+  float* logits_out;       // [T][E] or NULL
+  int32_t* idx;            // [T][k]
+  float* w;                // [T][k]
+  uint32_t* bitmap;        // [E][ceil(T/32)]
+  int* counter;            // one int, zero on entry
+  int32_t* offsets_r;      // [E+1] or NULL
+  int32_t* offsets_g;      // [E+2] or NULL
+  int32_t* chunk_prefix;   // [E+2] or NULL
+  int32_t* perm;           // [T*k]
+  int32_t* inv;            // [T*k]
+  int* active_out;         // += experts given rows, or NULL
+  int* err;
+};
+size_t router_smem_bytes(int T, int E);
+cudaError_t launch_router(const RouterArgs& a, cudaStream_t s);
 // xperm[T + p] = xperm[perm[p] / k] for p < k*T (rows [0, T) hold the normed input).
 cudaError_t launch_moe_gather(bf16* xperm, const int32_t* perm, int T, int k, int d,
                               cudaStream_t s);
@@ -132,7 +147,5 @@ cudaError_t launch_head_merge(const float* hm, const float* hs, const int* ha, i
 cudaError_t launch_commit(const float* conf, const int32_t* tok, int32_t* canvas,
                           uint8_t* committed, int B, int Tc, int steps_left,
                           const int* steps_left_dev, int mask_id, cudaStream_t s);
-cudaError_t launch_router_topk_only(const float* logits, int T, int E, int k, int32_t* idx,
-                                    float* w, uint32_t* bitmap, cudaStream_t s);
 
 }  // namespace dg

@@ -141,6 +141,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // everything above overlaps the previous kernel's tail; data access starts here
+  griddep_wait();
+  griddep_launch();
 
   const int n_tiles = tile_count(a);
   const int n_bufs = (a.mode == GEMM_HEAD) ? 1 : 2;
@@ -392,8 +395,8 @@ cudaError_t gemm_tc_launch(const CUtensorMap& mapA, const CUtensorMap& mapB, con
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  gemm_tc_kernel<<<grid, kThreads, gemm_smem_bytes(a), stream>>>(mapA, mapB, a);
-  return cudaGetLastError();
+  return launch_k(gemm_tc_kernel, dim3(grid), dim3(kThreads), gemm_smem_bytes(a), stream, mapA,
+                  mapB, a);
 }
 
 }  // namespace dg

@@ -1,0 +1,186 @@
+// Router: top-k expert selection per canvas row and the stable grouping of
+// the (row, slot) assignments by expert, in one kernel.
+//
+// One warp per row: the row's logits (split-K partials of the router GEMM,
+// summed in split order, plus the optional bias) are held 8 per lane; k rounds
+// of a warp-wide (value desc, index asc) argmax pick the experts; the weights
+// are the softmax over the chosen logits; each choice sets the row's bit in an
+// expert-membership bitmap.  The last block to finish (a device counter) then
+// runs a counting sort over the bitmap: per-expert counts, offsets, and each
+// assignment's position = offset + rows with the same expert before it.
+// Positions therefore follow row order inside an expert, with no float atomics.
+#include "dg_kernels.h"
+
+namespace dg {
+
+namespace {
+constexpr int kRouterThreads = 256;
+constexpr int kRowsPerBlock = kRouterThreads / 32;
+}  // namespace
+
+__global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
+  extern __shared__ int sm_dyn[];
+  __shared__ float s_sel_v[kRowsPerBlock][32];
+  __shared__ int s_sel_i[kRowsPerBlock][32];
+  __shared__ int s_last;
+  griddep_wait();
+  griddep_launch();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = a.T, E = a.E, k = a.k;
+  const int W = (T + 31) / 32;
+  const int t = blockIdx.x * kRowsPerBlock + warp;
+  if (t < T) {
+    // lane holds experts e = 128 * hh + 4 * lane + q
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    for (int s0 = 0; s0 < a.splits; s0 += 4) {
+      float4 buf[4][2];
+#pragma unroll
+      for (int ss = 0; ss < 4; ++ss)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int e0 = 128 * hh + 4 * lane;
+          if (s0 + ss < a.splits && e0 < E)
+            buf[ss][hh] = __ldg(reinterpret_cast<const float4*>(
+                a.logits_in + ((size_t)(s0 + ss) * T + t) * E + e0));
+        }
+#pragma unroll
+      for (int ss = 0; ss < 4; ++ss)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int e0 = 128 * hh + 4 * lane;
+          if (s0 + ss < a.splits && e0 < E) {
+            v[4 * hh + 0] += buf[ss][hh].x; v[4 * hh + 1] += buf[ss][hh].y;
+            v[4 * hh + 2] += buf[ss][hh].z; v[4 * hh + 3] += buf[ss][hh].w;
+          }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = 128 * (i >> 2) + 4 * lane + (i & 3);
+      float x = -INFINITY;
+      if (e < E) {
+        x = v[i] + (a.bias ? a.bias[e] : 0.f);
+        if (a.logits_out) a.logits_out[(size_t)t * E + e] = x;
+        if (x != x) x = -INFINITY;
+      }
+      v[i] = x;
+    }
+    unsigned taken = 0;
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = 128 * (i >> 2) + 4 * lane + (i & 3);
+        if (e < E && !(taken & (1u << i)) && (v[i] > bv || (v[i] == bv && e < bi))) {
+          bv = v[i];
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      }
+      if (bi >= 0 && bi < E && ((bi & 127) >> 2) == lane)
+        taken |= 1u << (4 * (bi >> 7) + (bi & 3));
+      if (lane == 0) {
+        s_sel_v[warp][j] = bv;
+        s_sel_i[warp][j] = bi;
+      }
+    }
+    __syncwarp();
+    if (lane < k) {
+      const float mx = s_sel_v[warp][0];
+      float den = 0.f;
+      for (int j = 0; j < k; ++j) den += __expf(s_sel_v[warp][j] - mx);
+      int e = s_sel_i[warp][lane];
+      if (e < 0 || e >= E) { raise_error(a.err, kErrFault); e = 0; }
+      a.idx[(size_t)t * k + lane] = e;
+      a.w[(size_t)t * k + lane] = __expf(s_sel_v[warp][lane] - mx) / den;
+      atomicOr(a.bitmap + (size_t)e * W + (t >> 5), 1u << (t & 31));
+    }
+  }
+
+  // ------------------------------------------------ the last block sorts
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(a.counter, 1) == (int)gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  int* prefix = sm_dyn;          // [E * W]
+  int* count = sm_dyn + E * W;   // [E]
+  int* off = count + E;          // [E + 1]
+  for (int i = threadIdx.x; i < E * W; i += blockDim.x) prefix[i] = __popc(__ldcg(a.bitmap + i));
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < W; ++w) {
+      const int c = prefix[e * W + w];
+      prefix[e * W + w] = run;
+      run += c;
+    }
+    count[e] = run;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    int crun = a.n_shared ? (T + a.n_tile - 1) / a.n_tile : 0;
+    if (a.offsets_g) a.offsets_g[0] = 0;
+    if (a.chunk_prefix) { a.chunk_prefix[0] = 0; a.chunk_prefix[1] = crun; }
+    int active = 0;
+    for (int e = 0; e < E; ++e) {
+      off[e] = run;
+      if (a.offsets_r) a.offsets_r[e] = run;
+      if (a.offsets_g) a.offsets_g[e + 1] = T + run;
+      run += count[e];
+      active += count[e] > 0;
+      crun += (count[e] + a.n_tile - 1) / a.n_tile;
+      if (a.chunk_prefix) a.chunk_prefix[e + 2] = crun;
+    }
+    off[E] = run;
+    if (a.offsets_r) a.offsets_r[E] = run;
+    if (a.offsets_g) a.offsets_g[E + 1] = T + run;
+    if (a.active_out) atomicAdd(a.active_out, active);
+    if (run != T * k) raise_error(a.err, kErrFault);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
+    const int tt = i / k;
+    const int e = __ldcg(a.idx + i);
+    if (e < 0 || e >= E) continue;
+    const uint32_t word = __ldcg(a.bitmap + (size_t)e * W + (tt >> 5));
+    const int pos = off[e] + prefix[e * W + (tt >> 5)] + __popc(word & ((1u << (tt & 31)) - 1u));
+    a.perm[pos] = i;
+    a.inv[i] = pos;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < E * W; i += blockDim.x) a.bitmap[i] = 0u;
+  if (threadIdx.x == 0) *a.counter = 0;
+}
+
+size_t router_smem_bytes(int T, int E) {
+  const int W = (T + 31) / 32;
+  return (size_t)(E * W + E + E + 1) * sizeof(int);
+}
+
+cudaError_t launch_router(const RouterArgs& a, cudaStream_t s) {
+  const size_t smem = router_smem_bytes(a.T, a.E);
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         200 * 1024);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  return launch_k(router_kernel, dim3((a.T + kRowsPerBlock - 1) / kRowsPerBlock),
+                  dim3(kRouterThreads), smem, s, a);
+}
+
+}  // namespace dg

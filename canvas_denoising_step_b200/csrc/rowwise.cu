@@ -1,0 +1,527 @@
+// Row-wise kernels of the canvas step: embedding + input norm, q/k RoPE,
+// post-attention norm + residual + pre-FFN norm, MoE gather and combine,
+// vocab-head merge and commit.
+//
+// Each row kernel runs one CTA of 256 threads per canvas row.  Thread i owns
+// the 8-element chunks i and i + 256 of the row (d <= 4096), loaded as 16-byte
+// vectors; the loads of several source rows (split-K partials, expert rows)
+// are issued together before any of them is used, so a CTA keeps tens of KB in
+// flight instead of one dependent round trip per source row.
+#include <cstdlib>
+
+#include "dg_kernels.h"
+
+namespace dg {
+
+namespace {
+
+constexpr int kRowThreads = 256;
+constexpr int kChunks = 2;  // 8-element chunks per thread: d <= 256 * 2 * 8
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int i = 0; i < kRowThreads / 32; ++i) t += red[i];
+  return t;
+}
+
+__device__ __forceinline__ void ld8f(const float* p, float* v) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// plain (coherent) loads for buffers written earlier in the same kernel chain
+__device__ __forceinline__ void ld8f_rw(const float* p, float* v) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0];
+  const float4 b = reinterpret_cast<const float4*>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+__device__ __forceinline__ void st8f(float* p, const float* v) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+__device__ __forceinline__ void ld8b(const bf16* p, float* v) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ void st8b(bf16* p, const float* v) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&b);
+  }
+  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+}  // namespace
+
+bool pdl_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("DG_NO_PDL");
+    v = (e && e[0] && e[0] != '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
+// ---------------------------------------------------------------- embed + input norm
+
+__global__ void __launch_bounds__(kRowThreads) embed_norm_kernel(
+    const int32_t* canvas, const bf16* embed, const bf16* x_in, int vocab, int d, const float* w,
+    float eps, float* h, bf16* x, int* err) {
+  __shared__ float red[32];
+  griddep_wait();
+  griddep_launch();
+  const int t = blockIdx.x;
+  const bf16* src;
+  if (x_in) {
+    src = x_in + (size_t)t * d;
+  } else {
+    int tok = canvas[t];
+    if (tok < 0 || tok >= vocab) { raise_error(err, kErrFault); tok = 0; }
+    src = embed + (size_t)tok * d;
+  }
+  const int n8 = d / 8;
+  float v[kChunks][8];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i) {
+    const int c = threadIdx.x + kRowThreads * i;
+    if (c < n8) ld8b(src + 8 * c, v[i]);
+    else
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[i][e] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss += v[i][e] * v[i][e];
+  }
+  ss = block_sum(ss, red);
+  const float r = rsqrtf(ss / (float)d + eps);
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i) {
+    const int c = threadIdx.x + kRowThreads * i;
+    if (c >= n8) continue;
+    float wv[8], o[8];
+    ld8f(w + 8 * c, wv);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = v[i][e] * r * wv[e];
+    st8f(h + (size_t)t * d + 8 * c, v[i]);
+    st8b(x + (size_t)t * d + 8 * c, o);
+  }
+}
+
+cudaError_t launch_embed_norm(const int32_t* canvas, const bf16* embed, const bf16* x_in,
+                              int vocab, int T, int d, const float* w, float eps, float* h,
+                              bf16* x, int* err, cudaStream_t s) {
+  return launch_k(embed_norm_kernel, dim3(T), dim3(kRowThreads), 0, s, canvas, embed, x_in,
+                  vocab, d, w, eps, h, x, err);
+}
+
+// ---------------------------------------------------------------- RoPE table
+
+__global__ void rope_table_kernel(float* cos_t, float* sin_t, int Tc, int half, int P,
+                                  double theta) {
+  griddep_wait();
+  griddep_launch();
+  const int id = blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= Tc * half) return;
+  const int i = id / half, j = id % half;
+  const double inv_freq = pow(theta, -2.0 * (double)j / (double)(2 * half));
+  const double ang = (double)(P + i) * inv_freq;
+  double sn, cs;
+  sincos(ang, &sn, &cs);
+  cos_t[id] = (float)cs;
+  sin_t[id] = (float)sn;
+}
+
+cudaError_t launch_rope_table(float* cos_t, float* sin_t, int Tc, int half, int P, double theta,
+                              cudaStream_t s) {
+  const int n = Tc * half;
+  return launch_k(rope_table_kernel, dim3((n + 255) / 256), dim3(256), 0, s, cos_t, sin_t, Tc,
+                  half, P, theta);
+}
+
+// ---------------------------------------------------------------- q/k/v split-K sum + RoPE
+
+// One CTA per canvas row.  Work item p = (head hh, 4-pair group j4): pairs
+// (j, j + dh/2) for j = 4*j4 .. 4*j4+3, loaded as two float4 per split.
+constexpr int kRopeItems = 8;  // items per thread: (Hq + 2 Hkv) * dh / 8 <= 2048
+
+__global__ void __launch_bounds__(kRowThreads) qkv_rope_kernel(
+    const float* part, int splits, int T, int Tc, int Hq, int Hkv, int dh, int n_rot,
+    const float* cos_t, const float* sin_t, bf16* q, bf16* kc, bf16* vc) {
+  griddep_wait();
+  griddep_launch();
+  const int t = blockIdx.x;
+  const int b = t / Tc, i = t % Tc;
+  const int nqkv = (Hq + 2 * Hkv) * dh;
+  const int half = dh / 2, q4 = half / 4;
+  const int n_items = (Hq + 2 * Hkv) * q4;
+  float4 x0[kRopeItems], x1[kRopeItems];
+#pragma unroll
+  for (int u = 0; u < kRopeItems; ++u) x0[u] = x1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < splits; ++s) {
+    const float* src = part + ((size_t)s * T + t) * nqkv;
+    float4 a[kRopeItems], c[kRopeItems];
+#pragma unroll
+    for (int u = 0; u < kRopeItems; ++u) {
+      const int p = threadIdx.x + kRowThreads * u;
+      if (p < n_items) {
+        const int hh = p / q4, j = (p % q4) * 4;
+        a[u] = __ldg(reinterpret_cast<const float4*>(src + hh * dh + j));
+        c[u] = __ldg(reinterpret_cast<const float4*>(src + hh * dh + j + half));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kRopeItems; ++u) {
+      x0[u].x += a[u].x; x0[u].y += a[u].y; x0[u].z += a[u].z; x0[u].w += a[u].w;
+      x1[u].x += c[u].x; x1[u].y += c[u].y; x1[u].z += c[u].z; x1[u].w += c[u].w;
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kRopeItems; ++u) {
+    const int p = threadIdx.x + kRowThreads * u;
+    if (p >= n_items) continue;
+    const int hh = p / q4, j = (p % q4) * 4;
+    bf16* dst;
+    bool rotate = true;
+    if (hh < Hq) dst = q + (((size_t)b * Hq + hh) * Tc + i) * dh;
+    else if (hh < Hq + Hkv) dst = kc + (((size_t)b * Hkv + (hh - Hq)) * Tc + i) * dh;
+    else { dst = vc + (((size_t)b * Hkv + (hh - Hq - Hkv)) * Tc + i) * dh; rotate = false; }
+    float lo[4] = {x0[u].x, x0[u].y, x0[u].z, x0[u].w};
+    float hi[4] = {x1[u].x, x1[u].y, x1[u].z, x1[u].w};
+    if (rotate) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (j + e < n_rot) {
+          const float cs = cos_t[i * half + j + e], sn = sin_t[i * half + j + e];
+          const float y0 = lo[e] * cs - hi[e] * sn;
+          const float y1 = lo[e] * sn + hi[e] * cs;
+          lo[e] = y0;
+          hi[e] = y1;
+        }
+      }
+    }
+    __nv_bfloat162 l01 = __floats2bfloat162_rn(lo[0], lo[1]), l23 = __floats2bfloat162_rn(lo[2], lo[3]);
+    __nv_bfloat162 h01 = __floats2bfloat162_rn(hi[0], hi[1]), h23 = __floats2bfloat162_rn(hi[2], hi[3]);
+    *reinterpret_cast<uint2*>(dst + j) =
+        make_uint2(*reinterpret_cast<uint32_t*>(&l01), *reinterpret_cast<uint32_t*>(&l23));
+    *reinterpret_cast<uint2*>(dst + j + half) =
+        make_uint2(*reinterpret_cast<uint32_t*>(&h01), *reinterpret_cast<uint32_t*>(&h23));
+  }
+}
+
+cudaError_t launch_qkv_rope(const float* part, int splits, int T, int Tc, int Hq, int Hkv, int dh,
+                            int n_rot, const float* cos_t, const float* sin_t, bf16* q, bf16* kc,
+                            bf16* vc, cudaStream_t s) {
+  return launch_k(qkv_rope_kernel, dim3(T), dim3(kRowThreads), 0, s, part, splits, T, Tc, Hq, Hkv,
+                  dh, n_rot, cos_t, sin_t, q, kc, vc);
+}
+
+// ---------------------------------------------------------------- post-attention norms
+
+__global__ void __launch_bounds__(kRowThreads) post_attn_kernel(
+    const float* part, int splits, int T, int d, const float* w_post, const float* w_ff, float eps,
+    float* h, bf16* x2) {
+  __shared__ float red[32];
+  griddep_wait();
+  griddep_launch();
+  const int t = blockIdx.x, n8 = d / 8;
+  float a[kChunks][8];
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) a[i][e] = 0.f;
+  for (int s0 = 0; s0 < splits; s0 += 4) {  // four splits' loads in flight at once
+    float buf[4][kChunks][8];
+#pragma unroll
+    for (int ss = 0; ss < 4; ++ss)
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        const int c = threadIdx.x + kRowThreads * i;
+        if (s0 + ss < splits && c < n8) ld8f(part + ((size_t)(s0 + ss) * T + t) * d + 8 * c, buf[ss][i]);
+      }
+#pragma unroll
+    for (int ss = 0; ss < 4; ++ss)
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        const int c = threadIdx.x + kRowThreads * i;
+        if (s0 + ss < splits && c < n8)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) a[i][e] += buf[ss][i][e];
+      }
+  }
+  float ss1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss1 += a[i][e] * a[i][e];
+  ss1 = block_sum(ss1, red);
+  const float r1 = rsqrtf(ss1 / (float)d + eps);
+  float ss2 = 0.f;
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i) {
+    const int c = threadIdx.x + kRowThreads * i;
+    if (c >= n8) continue;
+    float hv[8], wv[8];
+    ld8f_rw(h + (size_t)t * d + 8 * c, hv);
+    ld8f(w_post + 8 * c, wv);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      a[i][e] = hv[e] + a[i][e] * r1 * wv[e];
+      ss2 += a[i][e] * a[i][e];
+    }
+    st8f(h + (size_t)t * d + 8 * c, a[i]);
+  }
+  ss2 = block_sum(ss2, red);
+  const float r2 = rsqrtf(ss2 / (float)d + eps);
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i) {
+    const int c = threadIdx.x + kRowThreads * i;
+    if (c >= n8) continue;
+    float wv[8], o[8];
+    ld8f(w_ff + 8 * c, wv);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = a[i][e] * r2 * wv[e];
+    st8b(x2 + (size_t)t * d + 8 * c, o);
+  }
+}
+
+cudaError_t launch_post_attn(const float* part, int splits, int T, int d, const float* w_post,
+                             const float* w_ff, float eps, float* h, bf16* x2, cudaStream_t s) {
+  return launch_k(post_attn_kernel, dim3(T), dim3(kRowThreads), 0, s, part, splits, T, d, w_post,
+                  w_ff, eps, h, x2);
+}
+
+// ---------------------------------------------------------------- MoE gather / combine
+
+__global__ void moe_gather_kernel(bf16* xperm, const int32_t* perm, int T, int k, int d) {
+  griddep_wait();
+  griddep_launch();
+  const int p = blockIdx.x;
+  const int t = perm[p] / k;
+  const uint4* src = reinterpret_cast<const uint4*>(xperm + (size_t)t * d);
+  uint4* dst = reinterpret_cast<uint4*>(xperm + ((size_t)T + p) * d);
+  for (int i = threadIdx.x; i < d / 8; i += blockDim.x) dst[i] = src[i];
+}
+
+cudaError_t launch_moe_gather(bf16* xperm, const int32_t* perm, int T, int k, int d,
+                              cudaStream_t s) {
+  return launch_k(moe_gather_kernel, dim3(T * k), dim3(128), 0, s, xperm, perm, T, k, d);
+}
+
+// y_t = sum_{j < k} w_tj Y[T + inv(t,j)] (+ Y[t] for the shared expert), added in
+// the fixed order j = 0 .. k-1 then shared; h += y; then the next norm.
+__global__ void __launch_bounds__(kRowThreads) moe_combine_kernel(
+    const float* Y, const float* w, const int32_t* inv, int T, int k, int n_shared, int d, float* h,
+    const float* w_next, float eps, bf16* x) {
+  __shared__ float red[32];
+  __shared__ int srow[33];
+  __shared__ float sw[33];
+  griddep_wait();
+  griddep_launch();
+  const int t = blockIdx.x, n8 = d / 8;
+  if (threadIdx.x < k) {
+    srow[threadIdx.x] = T + inv[(size_t)t * k + threadIdx.x];
+    sw[threadIdx.x] = w[(size_t)t * k + threadIdx.x];
+  }
+  if (threadIdx.x == 0 && n_shared) {
+    srow[k] = t;
+    sw[k] = 1.0f;
+  }
+  __syncthreads();
+  const int nrows = k + (n_shared ? 1 : 0);
+  float y[kChunks][8];
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[i][e] = 0.f;
+  for (int j0 = 0; j0 < nrows; j0 += 4) {     // four source rows' loads in flight at once
+    float buf[4][kChunks][8];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        const int c = threadIdx.x + kRowThreads * i;
+        if (j0 + jj < nrows && c < n8) ld8f_rw(Y + (size_t)srow[j0 + jj] * d + 8 * c, buf[jj][i]);
+      }
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      if (j0 + jj >= nrows) break;
+      const float wj = sw[j0 + jj];
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        const int c = threadIdx.x + kRowThreads * i;
+        if (c < n8)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) y[i][e] += wj * buf[jj][i][e];
+      }
+    }
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i) {
+    const int c = threadIdx.x + kRowThreads * i;
+    if (c >= n8) continue;
+    float hv[8];
+    ld8f_rw(h + (size_t)t * d + 8 * c, hv);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      y[i][e] += hv[e];
+      ss += y[i][e] * y[i][e];
+    }
+    st8f(h + (size_t)t * d + 8 * c, y[i]);
+  }
+  if (w_next) {
+    ss = block_sum(ss, red);
+    const float r = rsqrtf(ss / (float)d + eps);
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+      const int c = threadIdx.x + kRowThreads * i;
+      if (c >= n8) continue;
+      float wv[8], o[8];
+      ld8f(w_next + 8 * c, wv);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = y[i][e] * r * wv[e];
+      st8b(x + (size_t)t * d + 8 * c, o);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+      const int c = threadIdx.x + kRowThreads * i;
+      if (c < n8) st8b(x + (size_t)t * d + 8 * c, y[i]);
+    }
+  }
+}
+
+cudaError_t launch_moe_combine(const float* Y, const float* w, const int32_t* inv, int T, int k,
+                               int n_shared, int d, float* h, const float* w_next, float eps,
+                               bf16* x, cudaStream_t s) {
+  return launch_k(moe_combine_kernel, dim3(T), dim3(kRowThreads), 0, s, Y, w, inv, T, k, n_shared,
+                  d, h, w_next, eps, x);
+}
+
+// ---------------------------------------------------------------- vocab head merge
+
+namespace {
+__device__ __forceinline__ void merge_stats(float& m, float& s, int& a, float m2, float s2,
+                                            int a2) {
+  if (m2 == -INFINITY) return;
+  if (m == -INFINITY) { m = m2; s = s2; a = a2; return; }
+  if (m2 > m) {
+    s = s * __expf(m - m2) + s2;
+    m = m2;
+    a = a2;
+  } else {
+    s = s + s2 * __expf(m2 - m);
+    if (m2 == m && a2 < a) a = a2;
+  }
+}
+}  // namespace
+
+__global__ void head_merge_kernel(const float* hm, const float* hs, const int* ha, int n_vblocks,
+                                  int T, float* conf, int32_t* tok) {
+  griddep_wait();
+  griddep_launch();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (t >= T) return;
+  float m = -INFINITY, s = 0.f;
+  int a = 0x7fffffff;
+  const int per = (n_vblocks + 31) / 32;
+  const int v0 = lane * per, v1 = min(n_vblocks, v0 + per);
+  for (int vb = v0; vb < v1; ++vb) {
+    const size_t o = (size_t)vb * T + t;
+    merge_stats(m, s, a, hm[o], hs[o], ha[o]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    const int a2 = __shfl_xor_sync(0xffffffffu, a, o);
+    merge_stats(m, s, a, m2, s2, a2);
+  }
+  if (lane == 0) {
+    conf[t] = 1.0f / s;
+    tok[t] = a;
+  }
+}
+
+cudaError_t launch_head_merge(const float* hm, const float* hs, const int* ha, int n_vblocks,
+                              int T, float* conf, int32_t* tok, cudaStream_t s) {
+  return launch_k(head_merge_kernel, dim3((T + 7) / 8), dim3(256), 0, s, hm, hs, ha, n_vblocks, T,
+                  conf, tok);
+}
+
+// ---------------------------------------------------------------- commit
+
+__global__ void commit_kernel(const float* conf, const int32_t* tok, int32_t* canvas,
+                              uint8_t* committed, int Tc, int steps_left, const int* steps_dev,
+                              int mask_id) {
+  __shared__ float sc[256];
+  __shared__ int sm[256];
+  griddep_wait();
+  griddep_launch();
+  const int b = blockIdx.x, i = threadIdx.x;
+  const size_t o = (size_t)b * Tc;
+  int masked = 0;
+  if (i < Tc) {
+    masked = canvas[o + i] == mask_id;
+    float c = conf[o + i];
+    if (c != c) c = -INFINITY;
+    sc[i] = c;
+    sm[i] = masked;
+  }
+  const int r = __syncthreads_count(masked);
+  const int sl = steps_left >= 1 ? steps_left : max(1, *steps_dev);
+  const int k = (r + sl - 1) / sl;
+  if (i < Tc) {
+    int com = 0;
+    if (masked) {
+      const float ci = sc[i];
+      int rank = 0;
+      for (int j = 0; j < Tc; ++j) rank += sm[j] && (sc[j] > ci || (sc[j] == ci && j < i));
+      if (rank < k) {
+        canvas[o + i] = tok[o + i];
+        com = 1;
+      }
+    }
+    if (committed) committed[o + i] = (uint8_t)com;
+  }
+}
+
+cudaError_t launch_commit(const float* conf, const int32_t* tok, int32_t* canvas,
+                          uint8_t* committed, int B, int Tc, int steps_left,
+                          const int* steps_left_dev, int mask_id, cudaStream_t s) {
+  return launch_k(commit_kernel, dim3(B), dim3(256), 0, s, conf, tok, canvas, committed, Tc,
+                  steps_left, steps_left_dev, mask_id);
+}
+
+}  // namespace dg
+
+namespace dg {
+
+__global__ void set_int_kernel(int* p, int v) { *p = v; }
+
+cudaError_t launch_set_int(int* p, int v, cudaStream_t s) {
+  set_int_kernel<<<1, 1, 0, s>>>(p, v);
+  return cudaGetLastError();
+}
+
+}  // namespace dg

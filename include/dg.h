@@ -68,7 +68,7 @@ typedef struct dg_ctx dg_ctx;
  *   d_model a multiple of 64 in [128, 4096]; d_ff a multiple of 64;
  *   head_dim in {64, 128, 256};
  *   n_q_heads a multiple of n_kv_heads; 1 <= top_k <= min(n_experts, 32);
- *   n_experts <= 256;
+ *   n_experts a multiple of 4 in [4, 256]; (n_q_heads + 2 n_kv_heads) * head_dim <= 16384;
  *   n_shared in {0, 1}; 1 <= canvas_len <= 256; max_batch * canvas_len <= 4096;
  *   0 <= mask_id < vocab; window >= 1; global_every >= 1.
  * Layer l (0-based) is global iff (l + 1) % global_every == 0: it attends to
@@ -153,7 +153,7 @@ int dg_layer_forward(dg_ctx* ctx, int layer, const void* x_in, void* x_out, int 
  * softmax over the chosen logits; offsets int32 [n_experts + 1]; perm int32
  * [n_rows * top_k] with perm[offsets[e] + r] = t * top_k + j for the r-th
  * assignment (t, j) to expert e in increasing t.  n_rows <= max_batch *
- * canvas_len. */
+ * canvas_len.  logits must be 16-byte aligned. */
 int dg_router_topk(dg_ctx* ctx, const float* logits, int n_rows, int32_t* idx, float* w,
                    int32_t* offsets, int32_t* perm);
 
@@ -202,7 +202,7 @@ int dg_profile_enable(dg_ctx* ctx, int on);
  * one kernel since dg_profile_enable(ctx, 1).  Synchronises.  Kernel names
  * are those returned by dg_kernel_name(0 ..): "embed_norm", "rope_table",
  * "gemm_qkv", "qkv_rope", "attention", "attn_merge", "gemm_o", "post_attn",
- * "gemm_router", "router_topk", "router_sort", "moe_gather", "gemm_gateup",
+ * "gemm_router", "router", "moe_gather", "gemm_gateup",
  * "gemm_down", "moe_combine", "gemm_head", "head_merge", "commit". */
 int dg_profile_read(dg_ctx* ctx, const char* kernel, double* total_ms, int* launches);
 

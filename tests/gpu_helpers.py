@@ -25,7 +25,11 @@ class Ctx:
         self.dg, self.cfg = dg, cfg
         self.B, self.Tc, self.P = cfg["batch"], cfg["canvas_len"], cfg["prompt_len"]
         self.T = self.B * self.Tc
-        self.stream = torch.cuda.current_stream().cuda_stream
+        # a dedicated stream (made current for torch too), so passes run from CUDA graphs
+        self.torch_stream = torch.cuda.Stream()
+        self.prev_stream = torch.cuda.current_stream()
+        torch.cuda.set_stream(self.torch_stream)
+        self.stream = self.torch_stream.cuda_stream
         self.ctx = dg.dg_create(dg.config_from_dict(cfg, max_batch, max_prompt), self.stream)
         dg.dg_init_weights(self.ctx, cfg["seed"])
         self.kv_host, self.kv_dev = [], []
@@ -47,6 +51,8 @@ class Ctx:
         if self.ctx:
             self.dg.dg_destroy(self.ctx)
             self.ctx = None
+            torch.cuda.synchronize()
+            torch.cuda.set_stream(self.prev_stream)
 
     def fetch(self, name: str, dtype, shape) -> np.ndarray:
         need = self.dg.dg_debug_tensor(self.ctx, name, None, 0)

@@ -291,6 +291,29 @@ def test_denoise_block_invariants_and_resume():
         c.close()
 
 
+def test_graph_and_direct_launch_agree(monkeypatch):
+    """Passes replayed from a captured CUDA graph give the same bits as direct launches."""
+    cfg = gpu_cfg("ragged")
+    results = []
+    for no_graph in ("0", "1"):
+        monkeypatch.setenv("DG_NO_GRAPH", no_graph)
+        c = Ctx(cfg)
+        try:
+            B, Tc, S = c.B, c.Tc, cfg["steps"]
+            can = synth.initial_canvas(cfg).cuda()
+            confs = []
+            for s in range(S):
+                conf = torch.empty(B, Tc, device="cuda")
+                c.dg.dg_canvas_step(c.ctx, can.data_ptr(), B, S - s, conf.data_ptr(), None)
+                confs.append(conf)
+            c.dg.dg_sync(c.ctx)
+            results.append((can.cpu().numpy(), torch.stack(confs).cpu().numpy()))
+        finally:
+            c.close()
+    assert np.array_equal(results[0][0], results[1][0])
+    assert np.array_equal(results[0][1], results[1][1])
+
+
 def test_host_buffer_step_matches_device_step():
     cfg = gpu_cfg("tiny")
     c = Ctx(cfg)
