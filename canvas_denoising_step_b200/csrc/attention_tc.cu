@@ -1,0 +1,345 @@
+// Canvas attention on the 5th-generation tensor cores (tcgen05).
+//
+// One softmax over {the visible prompt keys} U {all canvas keys} for every
+// canvas query row, with grouped-query heads.  A CTA takes 128 query rows of
+// one (canvas b, kv head g) -- the rows of the group's query heads, stacked --
+// and one contiguous range of 64-key blocks.  Prompt-key blocks and canvas-key
+// blocks are kept apart so that every block is one TMA box from one source.
+//
+// Roles (192 threads):
+//   warp 0, lane 0   TMA: the Q tile once, then K and V of each key block
+//                    into a two-stage ring (K and V share the layout
+//                    [dh/64][64 keys][128 B], 128-byte swizzle);
+//   warp 1           TMEM allocation; lane 0 issues the MMAs:
+//                    S_j = Q K_j^T into one of two S buffers (M=128, N=64),
+//                    then O += P_{j-1} V_{j-1} (M=128, N=dh, V as an MN-major
+//                    operand) once the softmax has written P_{j-1};
+//   warps 2..5       softmax, one query row per thread: read S_j from TMEM,
+//                    mask and scale (log2 units), keep a reference max m and
+//                    the running sum l; when a block's max exceeds m by more
+//                    than 8 (a factor 256) O is rescaled in TMEM, otherwise the
+//                    stale m is kept (P <= 256 stays exact enough in bf16);
+//                    write P_j as bf16 into shared memory in the K-major
+//                    128-byte-swizzle layout the MMA reads.
+// The CTA writes the un-normalised partial (O, m, l) of its key range; the
+// log-sum-exp merge kernel combines the ranges.
+#include "dg_kernels.h"
+
+namespace dg {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kBN = 64;          // keys per block
+constexpr int kRows = 128;       // query rows per CTA
+constexpr int kStages = 2;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int DH>
+struct AttnSmem {
+  static constexpr int kQ = kRows * DH * 2;         // Q tile
+  static constexpr int kKV = kBN * DH * 2;          // one K (or V) block
+  static constexpr int kP = kRows * kBN * 2;        // P tile
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQ;                  // [stage] K
+  static constexpr int kVOff = kKOff + kStages * kKV;
+  static constexpr int kPOff = kVOff + kStages * kKV;
+  static constexpr int kBarOff = kPOff + kP;
+  static constexpr int kBytes = kBarOff + 256;
+};
+
+}  // namespace
+
+template <int DH>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapKc,
+               const __grid_constant__ CUtensorMap mapVc, const __grid_constant__ CUtensorMap mapKp,
+               const __grid_constant__ CUtensorMap mapVp, const AttnTcArgs a) {
+  using L = AttnSmem<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bars = sbase + L::kBarOff;
+  // barrier slots (8 bytes each)
+  const uint32_t q_full = bars + 0;
+  auto kv_full = [&](int s) { return bars + 8u * (1 + s); };
+  auto kv_empty = [&](int s) { return bars + 8u * (3 + s); };
+  auto s_full = [&](int s) { return bars + 8u * (5 + s); };
+  auto s_free = [&](int s) { return bars + 8u * (7 + s); };
+  const uint32_t p_full = bars + 8u * 9;
+  const uint32_t pv_done = bars + 8u * 10;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOff + 8 * 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kBarOff + 8 * 12 + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = blockIdx.x, chunk = blockIdx.y;
+  const int b = blockIdx.z / a.Hkv, g = blockIdx.z % a.Hkv;
+  const int group = a.Hq / a.Hkv;
+  const int q_rows = group * a.Tc;
+  const int nbp = (a.n_vis + kBN - 1) / kBN;            // prompt-key blocks
+  const int nbc = (a.Tc + kBN - 1) / kBN;               // canvas-key blocks
+  const int nb = nbp + nbc;
+  const int jb0 = (int)(((long long)chunk * nb) / a.n_chunks);
+  const int jb1 = (int)(((long long)(chunk + 1) * nb) / a.n_chunks);
+  const int n_local = jb1 - jb0;
+  constexpr uint32_t kTmemCols = (DH + 2 * kBN <= 256) ? 256 : 512;
+  constexpr uint32_t kOCol = 0, kSCol = DH;             // O at [0, DH), S buffers after it
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+      mbar_init(s_full(s), 1);
+      mbar_init(s_free(s), 4);
+    }
+    mbar_init(p_full, 4);
+    mbar_init(pv_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&mapQ);
+    tma_prefetch_desc(&mapKc);
+    tma_prefetch_desc(&mapVc);
+    tma_prefetch_desc(&mapKp);
+    tma_prefetch_desc(&mapVp);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_wait();
+  griddep_launch();
+
+  if (warp == 0) {
+    if (lane == 0 && n_local > 0) {
+      // ---------------------------------------------------------- TMA producer
+      const int q_row0 = (b * a.Hq + g * group) * a.Tc + qt * kRows;
+      mbar_arrive_expect_tx(q_full, (uint32_t)L::kQ);
+      for (int c = 0; c < DH / 64; ++c)
+        tma_load_2d(sbase + L::kQOff + c * (kRows * 128), &mapQ, q_full, c * 64, q_row0);
+      bool ok = true;
+      int issued = 0;
+      for (int j = 0; j < n_local && ok; ++j) {
+        const int st = j % kStages;
+        const uint32_t par = (uint32_t)((j / kStages) & 1) ^ 1u;
+        if (!mbar_wait(kv_empty(st), par, abort_flag, a.err)) { ok = false; break; }
+        const int jg = jb0 + j;
+        const CUtensorMap* mk;
+        const CUtensorMap* mv;
+        int row;
+        if (jg < nbp) {
+          mk = &mapKp; mv = &mapVp;
+          row = (b * a.Hkv + g) * a.P + (a.P - a.n_vis) + jg * kBN;
+        } else {
+          mk = &mapKc; mv = &mapVc;
+          row = (b * a.Hkv + g) * a.Tc + (jg - nbp) * kBN;
+        }
+        mbar_arrive_expect_tx(kv_full(st), (uint32_t)(2 * L::kKV));
+        for (int c = 0; c < DH / 64; ++c) {
+          tma_load_2d(sbase + L::kKOff + st * L::kKV + c * (kBN * 128), mk, kv_full(st), c * 64, row);
+          tma_load_2d(sbase + L::kVOff + st * L::kKV + c * (kBN * 128), mv, kv_full(st), c * 64, row);
+        }
+        ++issued;
+      }
+      if (!ok) {  // abort path: let issued copies land
+        mbar_drain(q_full, 0);
+        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+          mbar_drain(kv_full(j % kStages), (uint32_t)((j / kStages) & 1));
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && n_local > 0) {
+      // ---------------------------------------------------------- MMA issuer
+      const uint32_t idesc_s = idesc_bf16_f32(kBN);
+      const uint32_t idesc_o = idesc_bf16_f32(DH, false, true);   // B (= V) MN-major
+      bool ok = mbar_wait(q_full, 0, abort_flag, a.err);
+      tc_fence_after();
+      for (int j = 0; j <= n_local && ok; ++j) {
+        if (j < n_local) {
+          const int st = j % kStages, sb = j % 2;
+          if (!mbar_wait(kv_full(st), (uint32_t)((j / kStages) & 1), abort_flag, a.err)) { ok = false; break; }
+          if (!mbar_wait(s_free(sb), (uint32_t)((j / 2) & 1) ^ 1u, abort_flag, a.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kbase = sbase + L::kKOff + st * L::kKV;
+#pragma unroll
+          for (int kk = 0; kk < DH / 16; ++kk) {
+            const int c = kk >> 2, w = (kk & 3) * 32;
+            const uint64_t ad = sdesc_kmajor_sw128(sbase + L::kQOff + c * (kRows * 128) + w);
+            const uint64_t bd = sdesc_kmajor_sw128(kbase + c * (kBN * 128) + w);
+            umma_bf16(tmem + kSCol + sb * kBN, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(s_full(sb));
+        }
+        if (j >= 1) {
+          const int jp = j - 1, stp = jp % kStages;
+          if (!mbar_wait(p_full, (uint32_t)(jp & 1), abort_flag, a.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t vbase = sbase + L::kVOff + stp * L::kKV;
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            const uint64_t ad = sdesc_kmajor_sw128(sbase + L::kPOff + kk * 32);
+            const uint64_t bd = sdesc_mnmajor_sw128(vbase + kk * (16 * 128), kBN * 128);
+            umma_bf16(tmem + kOCol, ad, bd, idesc_o, (jp > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(pv_done);
+          umma_commit(kv_empty(stp));
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int q = warp & 3;
+    const int r = q * 32 + lane;                       // query row in the tile
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    uint32_t v[32];
+    for (int j = 0; j < n_local; ++j) {
+      const int sb = j % 2;
+      if (!mbar_wait(s_full(sb), (uint32_t)((j / 2) & 1), abort_flag, a.err)) { ok = false; break; }
+      tc_fence_after();
+      float s[kBN];
+#pragma unroll
+      for (int h = 0; h < kBN / 32; ++h) {
+        tmem_ld32(lane_base + kSCol + sb * kBN + h * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[h * 32 + e] = __uint_as_float(v[e]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free(sb));
+      // mask and scale
+      const int jg = jb0 + j;
+      const int valid = (jg < nbp) ? min(kBN, a.n_vis - jg * kBN) : min(kBN, a.Tc - (jg - nbp) * kBN);
+      float bmax = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < kBN; ++e) {
+        s[e] = (e < valid) ? s[e] * a.scale_log2 : -INFINITY;
+        bmax = fmaxf(bmax, s[e]);
+      }
+      // P_{j-1} consumed and O up to date before P_j or O is touched
+      if (j >= 1) {
+        if (!mbar_wait(pv_done, (uint32_t)((j - 1) & 1), abort_flag, a.err)) { ok = false; break; }
+        tc_fence_after();
+      }
+      if (m == -INFINITY) {
+        m = bmax;
+      } else if (bmax > m + kRescaleThreshold) {
+        const float f = exp2f(m - bmax);
+        l *= f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < DH; c0 += 32) {
+          tmem_ld32(lane_base + kOCol + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+          tmem_st32(lane_base + kOCol + c0, v);
+        }
+        tmem_wait_st();
+        m = bmax;
+      }
+      // P = 2^(s - m) as bf16, row r of the K-major swizzled tile
+      uint32_t pk[kBN / 2];
+#pragma unroll
+      for (int e = 0; e < kBN; e += 2) {
+        const float p0 = exp2f(s[e] - m), p1 = exp2f(s[e + 1] - m);
+        l += p0 + p1;
+        __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
+        pk[e / 2] = *reinterpret_cast<uint32_t*>(&bb);
+      }
+      uint8_t* prow = smem + L::kPOff + r * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int pc = c ^ (r & 7);
+        *reinterpret_cast<uint4*>(prow + pc * 16) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    // final O, then the partial of this key range
+    if (ok && n_local > 0) ok = mbar_wait(pv_done, (uint32_t)((n_local - 1) & 1), abort_flag, a.err);
+    tc_fence_after();
+    const int qr = qt * kRows + r;
+    const int rows_total = a.B * a.Hq * a.Tc;
+    const bool row_valid = qr < q_rows;
+    size_t R = 0;
+    if (row_valid) {
+      const int h = g * group + qr / a.Tc, i = qr % a.Tc;
+      R = ((size_t)b * a.Hq + h) * a.Tc + i;
+    }
+    float* po = a.part_o + ((size_t)chunk * rows_total + R) * DH;
+#pragma unroll 1
+    for (int c0 = 0; c0 < DH; c0 += 32) {
+      if (n_local > 0 && ok) {
+        tmem_ld32(lane_base + kOCol + c0, v);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = 0u;
+      }
+      if (row_valid) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(po + c0 + e) =
+              make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                          __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+      }
+    }
+    if (row_valid) {
+      float* pml = a.part_ml + ((size_t)chunk * rows_total + R) * 2;
+      pml[0] = (n_local > 0) ? m : -INFINITY;
+      pml[1] = l;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+namespace {
+
+template <int DH>
+cudaError_t launch_attn_tc_t(const AttnTcMaps& m, const AttnTcArgs& a, cudaStream_t s) {
+  const size_t smem = AttnSmem<DH>::kBytes + 1024;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DH>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int group = a.Hq / a.Hkv;
+  dim3 grid((group * a.Tc + kRows - 1) / kRows, a.n_chunks, a.B * a.Hkv);
+  return launch_k(attn_tc_kernel<DH>, grid, dim3(kThreads), smem, s, m.q, m.kc, m.vc, m.kp, m.vp, a);
+}
+
+}  // namespace
+
+int attn_tc_blocks(int n_vis, int Tc) { return (n_vis + kBN - 1) / kBN + (Tc + kBN - 1) / kBN; }
+int attn_tc_qtiles(int Hq, int Hkv, int Tc) { return (Hq / Hkv * Tc + kRows - 1) / kRows; }
+
+cudaError_t launch_attention_tc(const AttnTcMaps& m, const AttnTcArgs& a, cudaStream_t s) {
+  switch (a.dh) {
+    case 64: return launch_attn_tc_t<64>(m, a, s);
+    case 128: return launch_attn_tc_t<128>(m, a, s);
+    case 256: return launch_attn_tc_t<256>(m, a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace dg

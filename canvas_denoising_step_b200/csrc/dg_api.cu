@@ -26,6 +26,7 @@ struct Layer {
   bf16 *wqkv = nullptr, *wo = nullptr, *wr = nullptr, *wgu = nullptr, *wd = nullptr;
   float *ln_in = nullptr, *ln_post = nullptr, *ln_ff = nullptr;
   CUtensorMap m_qkv, m_o, m_r, m_gu, m_d;
+  CUtensorMap m_kp, m_vp;   // prompt K/V of this layer, 64-row boxes
   const bf16* kp = nullptr;
   const bf16* vp = nullptr;
   int kv_batch = 0, kv_P = 0;
@@ -79,6 +80,7 @@ struct dg_ctx {
   float* router_bias = nullptr;
   bool has_bias = false;
   CUtensorMap m_x_b, m_x_a, m_attn_o_b, m_xperm_b, m_H_b;
+  CUtensorMap m_q, m_kc, m_vc;   // attention operands
 
   int last_T = 0, last_B = 0, launches = 0;
   int* steps_dev = nullptr;          // steps_left of the pass being run
@@ -219,7 +221,9 @@ int run_dense(dg_ctx* c, int kind, const CUtensorMap& mA, const CUtensorMap& mB,
   a.mode = GEMM_DENSE;
   a.M = M; a.N = N; a.K = K; a.n_kb = K / 64;
   a.n_tile = std::min(256, (N + 31) / 32 * 32);
-  a.m_slabs = (M + 127) / 128;
+  // wide activation tiles: pair two weight slabs per tile to halve B traffic
+  a.dense_pair = (a.n_tile >= 128 && M > 128) ? 1 : 0;
+  a.m_slabs = (M + 128 * (1 + a.dense_pair) - 1) / (128 * (1 + a.dense_pair));
   const int n_chunks = (N + a.n_tile - 1) / a.n_tile;
   a.k_splits = choose_splits(a.m_slabs * n_chunks, a.n_kb, c->num_sms);
   if ((size_t)a.k_splits * N * M > c->part_elems) a.k_splits = 1;
@@ -272,21 +276,27 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
                                c->rope_sin, c->q, c->kc, c->vc, c->stream));
 
   // one softmax over the visible prompt keys and all canvas keys, split-KV
-  AttnArgs at;
+  AttnTcArgs ta;
+  memset(&ta, 0, sizeof(ta));
+  ta.B = B; ta.Hq = Hq; ta.Hkv = Hkv; ta.Tc = Tc; ta.P = P; ta.dh = dh;
+  ta.n_vis = is_global(cf, l) ? P : std::min(cf.window, P);
+  {
+    // key-block ranges per (canvas, kv head, query tile): about one CTA per SM
+    const int nb = attn_tc_blocks(ta.n_vis, Tc);
+    const int base = attn_tc_qtiles(Hq, Hkv, Tc) * B * Hkv;
+    ta.n_chunks = std::max(1, std::min({kMaxAttnChunks, nb, c->num_sms / base}));
+  }
+  ta.part_o = c->attn_po; ta.part_ml = c->attn_ml;
+  ta.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)dh));
+  ta.err = c->err_dev;
+  AttnTcMaps tm;
+  tm.q = c->m_q; tm.kc = c->m_kc; tm.vc = c->m_vc; tm.kp = L.m_kp; tm.vp = L.m_vp;
+  DG_LAUNCH(c, K_ATTN, launch_attention_tc(tm, ta, c->stream));
+  AttnArgs at;   // the merge reads the partials' shape from here
   memset(&at, 0, sizeof(at));
-  at.q = c->q; at.kc = c->kc; at.vc = c->vc; at.kp = L.kp; at.vp = L.vp;
   at.B = B; at.Hq = Hq; at.Hkv = Hkv; at.Tc = Tc; at.P = P; at.dh = dh;
-  at.n_vis = is_global(cf, l) ? P : std::min(cf.window, P);
-  const int NK = at.n_vis + Tc;
-  const int q_tiles = (Hq / Hkv * Tc + 63) / 64;
-  const int base = q_tiles * B * Hkv;
-  int nch = std::max(1, std::min(kMaxAttnChunks, (2 * c->num_sms + base - 1) / base));
-  nch = std::min(nch, (NK + 63) / 64);
-  at.chunk_keys = ((NK + nch - 1) / nch + 63) / 64 * 64;
-  at.n_chunks = (NK + at.chunk_keys - 1) / at.chunk_keys;
+  at.n_chunks = ta.n_chunks;
   at.part_o = c->attn_po; at.part_ml = c->attn_ml;
-  at.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)dh));
-  DG_LAUNCH(c, K_ATTN, launch_attention(at, c->stream));
   DG_LAUNCH(c, K_ATTN_MERGE, launch_attn_merge(at, c->attn_o, c->stream));
 
   // output projection, post-attention norm + residual, pre-FFN norm
@@ -499,9 +509,9 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
     ok &= alloc_n(c, &c->h, T * d);
     ok &= alloc_n(c, &c->x, Tp * d);
     ok &= alloc_n(c, &c->part, c->part_elems);
-    ok &= alloc_n(c, &c->q, T * Hq * dh);
-    ok &= alloc_n(c, &c->kc, T * Hkv * dh);
-    ok &= alloc_n(c, &c->vc, T * Hkv * dh);
+    ok &= alloc_n(c, &c->q, std::max<size_t>(T * Hq, 128) * dh);
+    ok &= alloc_n(c, &c->kc, std::max<size_t>(T * Hkv, 64) * dh);
+    ok &= alloc_n(c, &c->vc, std::max<size_t>(T * Hkv, 64) * dh);
     ok &= alloc_n(c, &c->attn_po, (size_t)kMaxAttnChunks * T * Hq * dh);
     ok &= alloc_n(c, &c->attn_ml, (size_t)kMaxAttnChunks * T * Hq * 2);
     ok &= alloc_n(c, &c->attn_o, Tp * Hq * dh);
@@ -549,6 +559,10 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
   cudaMemset(c->xperm, 0, rows_moe * d * 2);
   cudaMemset(c->H, 0, rows_moe * F * 2);
   cudaMemset(c->x, 0, Tp * d * 2);
+  // rows past T read by attention tiles must be finite (a masked key still multiplies V)
+  cudaMemset(c->q, 0, std::max<size_t>(T * Hq, 128) * dh * 2);
+  cudaMemset(c->kc, 0, std::max<size_t>(T * Hkv, 64) * dh * 2);
+  cudaMemset(c->vc, 0, std::max<size_t>(T * Hkv, 64) * dh * 2);
   cudaMemset(c->attn_o, 0, Tp * Hq * dh * 2);
   for (auto& L : c->layers) cudaMemset(L.wr, 0, Er * d * 2);
   // tensor maps (weights: A operands, 128-row boxes; activations: B operands, 32-row boxes)
@@ -565,6 +579,9 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
   ok &= make_tmap_2d(&c->m_attn_o_b, c->attn_o, (uint64_t)Hq * dh, Tp, 32);
   ok &= make_tmap_2d(&c->m_xperm_b, c->xperm, d, rows_moe, 32);
   ok &= make_tmap_2d(&c->m_H_b, c->H, F, rows_moe, 32);
+  ok &= make_tmap_2d(&c->m_q, c->q, dh, std::max<size_t>(T * Hq, 128), 128);
+  ok &= make_tmap_2d(&c->m_kc, c->kc, dh, std::max<size_t>(T * Hkv, 64), 64);
+  ok &= make_tmap_2d(&c->m_vc, c->vc, dh, std::max<size_t>(T * Hkv, 64), 64);
   if (cudaDeviceSynchronize() != cudaSuccess || !ok) {
     cudaGetLastError();
     free_all(c);
@@ -630,7 +647,13 @@ int dg_set_prompt_kv(dg_ctx* c, int layer, const void* k, const void* v, int bat
   if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15)
     return fail(c, DG_ERR_INVALID_ARG, "prompt K/V must be 16-byte aligned");
   Layer& L = c->layers[layer];
-  if (L.kp != k || L.vp != v || L.kv_batch != batch || L.kv_P != n_prompt) drop_graphs(c);
+  if (L.kp != k || L.vp != v || L.kv_batch != batch || L.kv_P != n_prompt) {
+    drop_graphs(c);
+    const uint64_t rows = (uint64_t)batch * c->cfg.n_kv_heads * n_prompt;
+    if (!make_tmap_2d(&L.m_kp, k, c->cfg.head_dim, rows, 64) ||
+        !make_tmap_2d(&L.m_vp, v, c->cfg.head_dim, rows, 64))
+      return fail(c, DG_ERR_CUDA, "tensor map for the prompt K/V failed");
+  }
   L.kp = static_cast<const bf16*>(k);
   L.vp = static_cast<const bf16*>(v);
   L.kv_batch = batch;

@@ -12,6 +12,7 @@ struct GemmArgs {
   int M, N, K, n_kb;      // A rows, B rows, reduction length, K / 64
   int n_tile;             // B rows per tile (DENSE / grouped)
   int k_splits;           // DENSE split-K
+  int dense_pair;         // DENSE: tiles of two 128-row slabs (m_slabs counts pairs)
   int m_slabs;            // 128-row slabs of A per group (DENSE / grouped)
   int n_groups;           // grouped: number of groups
   const int* offsets;     // grouped: [n_groups + 1] first B row of each group
@@ -95,6 +96,25 @@ struct AttnArgs {
   float scale_log2;  // log2(e) / sqrt(dh)
 };
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
+
+// tcgen05 attention (attention_tc.cu): same partial outputs as launch_attention.
+struct AttnTcArgs {
+  int B, Hq, Hkv, Tc, P, dh;
+  int n_vis;
+  int n_chunks;          // key-block ranges per (canvas, kv head, query tile)
+  float* part_o;         // [n_chunks][B*Hq*Tc][dh]
+  float* part_ml;        // [n_chunks][B*Hq*Tc][2]
+  float scale_log2;
+  int* err;
+};
+struct AttnTcMaps {
+  CUtensorMap q;         // [B*Hq*Tc][dh], box 64 x 128 rows
+  CUtensorMap kc, vc;    // [B*Hkv*Tc][dh], box 64 x 64 rows
+  CUtensorMap kp, vp;    // [B*Hkv*P][dh],  box 64 x 64 rows
+};
+int attn_tc_blocks(int n_vis, int Tc);
+int attn_tc_qtiles(int Hq, int Hkv, int Tc);
+cudaError_t launch_attention_tc(const AttnTcMaps& m, const AttnTcArgs& a, cudaStream_t s);
 // Merge partials -> o [T][Hq*dh] bf16 (t = b*Tc + i)
 cudaError_t launch_attn_merge(const AttnArgs& a, bf16* o, cudaStream_t s);
 

@@ -12,7 +12,8 @@
 // activation rows are N), and the token rows for the vocab head.
 //
 // Modes
-//  DENSE   Y[s][n][m] = sum_{k in split s} X[n][k] W[m][k]      (fp32 split-K partials)
+//  DENSE   Y[s][n][m] = sum_{k in split s} X[n][k] W[m][k]      (fp32 split-K partials);
+//          with dense_pair a tile holds two 128-row weight slabs sharing one B tile
 //  GATEUP  H[r][f] = silu(g) * u, with g/u the gate/up rows 2f/2f+1 of the
 //          group's interleaved weight, for rows r of the group     (bf16)
 //  DOWN    Y[r][m] = sum_k H[r][k] Wd[g][m][k]                   (fp32)
@@ -31,9 +32,11 @@ constexpr int kATileBytes = 128 * 128;  // 128 rows x 128 B
 
 struct TileInfo {
   int g, m_slab, row0, rows, kb0, kb1, split, tb, vb;
+  int a_row0;  // first A row of the tile (accumulator i covers a_row0 + 128 i ..)
   int n_acc;   // accumulators (A tiles) per tile
   int n_mma;   // MMA N
   int n_bbox;  // B boxes per stage
+  int rot;     // the k-blocks run in the order kb0 + (rot + i) % (kb1 - kb0)
 };
 
 __device__ __forceinline__ int upper_bound_prefix(const int* prefix, int n, int c) {
@@ -68,6 +71,8 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t) {
     ti.rows = min(a.n_tile, a.N - ti.row0);
     ti.kb0 = (int)(((long long)ti.split * a.n_kb) / a.k_splits);
     ti.kb1 = (int)(((long long)(ti.split + 1) * a.n_kb) / a.k_splits);
+    ti.n_acc = a.dense_pair ? 2 : 1;
+    ti.a_row0 = ti.m_slab * 128 * ti.n_acc;
   } else if (a.mode == GEMM_GATEUP || a.mode == GEMM_DOWN) {
     ti.m_slab = t % a.m_slabs;
     const int c = t / a.m_slabs;
@@ -78,6 +83,7 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t) {
     ti.rows = min(a.n_tile, end - ti.row0);
     ti.kb0 = 0;
     ti.kb1 = a.n_kb;
+    ti.a_row0 = ti.m_slab * 128;
   } else {  // HEAD
     ti.tb = t % a.n_tblocks;
     ti.vb = t / a.n_tblocks;
@@ -87,7 +93,12 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t) {
     ti.n_acc = (a.T - ti.tb * 256 > 128) ? 2 : 1;
     ti.kb0 = 0;
     ti.kb1 = a.n_kb;
+    ti.a_row0 = ti.tb * 256;
   }
+  // Tiles that run at the same time and share an operand (the slabs of one
+  // projection or expert, the vocab blocks of the head) start their k loops at
+  // different blocks so they do not all read the same lines at once.
+  ti.rot = ((a.mode == GEMM_HEAD ? ti.vb : ti.m_slab) * 5) % max(1, ti.kb1 - ti.kb0);
   if (a.mode == GEMM_HEAD) {
     ti.n_mma = 256;
     ti.n_bbox = 1;
@@ -146,7 +157,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   griddep_launch();
 
   const int n_tiles = tile_count(a);
-  const int n_bufs = (a.mode == GEMM_HEAD) ? 1 : 2;
+  const int n_bufs = (a.mode == GEMM_HEAD || (a.mode == GEMM_DENSE && a.dense_pair)) ? 1 : 2;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -158,20 +169,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         const TileInfo ti = decode_tile(a, t);
         const uint32_t tx = (uint32_t)(ti.n_acc * kATileBytes) +
                             (uint32_t)(ti.n_bbox * a.b_box_rows * 128);
-        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+        const int nk = ti.kb1 - ti.kb0;
+        for (int ik = 0; ik < nk; ++ik) {
+          const int kb = ti.kb0 + (ti.rot + ik) % nk;
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.err)) { ok = false; break; }
           const uint32_t sA = smem_base + (uint32_t)stage * a.stage_bytes;
           const uint32_t sB = sA + (uint32_t)a.a_bytes;
           const uint32_t fb = full_bar(stage);
           mbar_arrive_expect_tx(fb, tx);
           const int kx = kb * kBK;
-          if (a.mode == GEMM_DENSE) {
-            tma_load_2d(sA, &mapA, fb, kx, ti.m_slab * 128);
-          } else if (a.mode == GEMM_HEAD) {
+          if (a.mode == GEMM_DENSE || a.mode == GEMM_HEAD) {
             for (int i = 0; i < ti.n_acc; ++i)
-              tma_load_2d(sA + i * kATileBytes, &mapA, fb, kx, ti.tb * 256 + i * 128);
+              tma_load_2d(sA + i * kATileBytes, &mapA, fb, kx, ti.a_row0 + i * 128);
           } else {
-            tma_load_3d(sA, &mapA, fb, kx, ti.m_slab * 128, ti.g);
+            tma_load_3d(sA, &mapA, fb, kx, ti.a_row0, ti.g);
           }
           for (int i = 0; i < ti.n_bbox; ++i)
             tma_load_2d(sB + (uint32_t)(i * a.b_box_rows * 128), &mapB, fb, kx,
@@ -202,7 +213,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         tc_fence_after();
         const uint32_t d_base = tmem_base + (uint32_t)buf * 256u;
         const uint32_t idesc = idesc_bf16_f32(ti.n_mma);
-        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+        const int nk = ti.kb1 - ti.kb0;
+        for (int ik = 0; ik < nk; ++ik) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sA = smem_base + (uint32_t)stage * a.stage_bytes;
@@ -213,7 +225,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
             for (int i = 0; i < ti.n_acc; ++i) {
               const uint64_t adesc = sdesc_kmajor_sw128(sA + i * kATileBytes + kk * 32);
               umma_bf16(d_base + (uint32_t)i * 256u, adesc, bdesc, idesc,
-                        (kb > ti.kb0 || kk > 0) ? 1u : 0u);
+                        (ik > 0 || kk > 0) ? 1u : 0u);
             }
           }
           umma_commit(empty_bar(stage));
@@ -238,16 +250,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)buf * 256u;
       uint32_t v[32];
       if (a.mode == GEMM_DENSE || a.mode == GEMM_DOWN) {
-        const int m = ti.m_slab * 128 + r;
         float* out = a.out_f32 + (size_t)ti.split * a.N * a.M;
-        for (int c0 = 0; c0 < ti.n_mma; c0 += 32) {
-          tmem_ld32(lane_addr + c0, v);
-          tmem_wait_ld();
-          if (m < a.M) {
+        for (int i = 0; i < ti.n_acc; ++i) {
+          const int m = ti.a_row0 + i * 128 + r;
+          for (int c0 = 0; c0 < ti.n_mma; c0 += 32) {
+            tmem_ld32(lane_addr + (uint32_t)i * 256u + c0, v);
+            tmem_wait_ld();
+            if (m < a.M) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int n = c0 + j;
-              if (n < ti.rows) out[(size_t)(ti.row0 + n) * a.M + m] = __uint_as_float(v[j]);
+              for (int j = 0; j < 32; ++j) {
+                const int n = c0 + j;
+                if (n < ti.rows) out[(size_t)(ti.row0 + n) * a.M + m] = __uint_as_float(v[j]);
+              }
             }
           }
         }
@@ -368,7 +382,7 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t m
 // Shared-memory plan: A region (1 or 2 tiles of 16 KB) + B region, as many
 // stages as fit in ~220 KB.
 void gemm_plan_smem(GemmArgs& a) {
-  const int n_a = (a.mode == GEMM_HEAD) ? 2 : 1;
+  const int n_a = (a.mode == GEMM_HEAD || (a.mode == GEMM_DENSE && a.dense_pair)) ? 2 : 1;
   a.a_bytes = n_a * kATileBytes;
   if (a.mode == GEMM_HEAD) {
     a.b_box_rows = 256;

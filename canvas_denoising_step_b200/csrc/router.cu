@@ -117,7 +117,12 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
   int* prefix = sm_dyn;          // [E * W]
   int* count = sm_dyn + E * W;   // [E]
   int* off = count + E;          // [E + 1]
-  for (int i = threadIdx.x; i < E * W; i += blockDim.x) prefix[i] = __popc(__ldcg(a.bitmap + i));
+  uint32_t* words = reinterpret_cast<uint32_t*>(off + E + 1);  // [E * W]
+  for (int i = threadIdx.x; i < E * W; i += blockDim.x) {
+    const uint32_t wv = __ldcg(a.bitmap + i);
+    words[i] = wv;
+    prefix[i] = __popc(wv);
+  }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int run = 0;
@@ -151,14 +156,24 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
     if (run != T * k) raise_error(a.err, kErrFault);
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
-    const int tt = i / k;
-    const int e = __ldcg(a.idx + i);
-    if (e < 0 || e >= E) continue;
-    const uint32_t word = __ldcg(a.bitmap + (size_t)e * W + (tt >> 5));
-    const int pos = off[e] + prefix[e * W + (tt >> 5)] + __popc(word & ((1u << (tt & 31)) - 1u));
-    a.perm[pos] = i;
-    a.inv[i] = pos;
+  for (int i0 = 0; i0 < T * k; i0 += 8 * kRouterThreads) {  // 8 index loads in flight per thread
+    int ev[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * kRouterThreads + threadIdx.x;
+      ev[u] = (i < T * k) ? __ldcg(a.idx + i) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * kRouterThreads + threadIdx.x;
+      const int e = ev[u];
+      if (i >= T * k || e < 0 || e >= E) continue;
+      const int tt = i / k;
+      const uint32_t word = words[e * W + (tt >> 5)];
+      const int pos = off[e] + prefix[e * W + (tt >> 5)] + __popc(word & ((1u << (tt & 31)) - 1u));
+      a.perm[pos] = i;
+      a.inv[i] = pos;
+    }
   }
   __syncthreads();
   for (int i = threadIdx.x; i < E * W; i += blockDim.x) a.bitmap[i] = 0u;
@@ -167,7 +182,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
 
 size_t router_smem_bytes(int T, int E) {
   const int W = (T + 31) / 32;
-  return (size_t)(E * W + E + E + 1) * sizeof(int);
+  return (size_t)(2 * E * W + E + E + 1) * sizeof(int);
 }
 
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t s) {
