@@ -83,8 +83,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
   const int jb0 = (int)(((long long)chunk * nb) / a.n_chunks);
   const int jb1 = (int)(((long long)(chunk + 1) * nb) / a.n_chunks);
   const int n_local = jb1 - jb0;
-  constexpr uint32_t kTmemCols = (DH + 2 * kBN <= 256) ? 256 : 512;
-  constexpr uint32_t kOCol = 0, kSCol = DH;             // O at [0, DH), S buffers after it
+  // TMEM: O at [0, DH); then two S buffers, each split into kSChains
+  // independent accumulator chains of kBN columns (the k16 steps of QK^T
+  // alternate between chains so consecutive MMAs do not depend on each other).
+  constexpr int kSChains = (DH + 2 * 4 * kBN <= 512) ? 4 : 2;
+  constexpr uint32_t kTmemCols = (DH + 2 * kSChains * kBN <= 256) ? 256 : 512;
+  constexpr uint32_t kOCol = 0, kSCol = DH;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -170,9 +174,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
 #pragma unroll
           for (int kk = 0; kk < DH / 16; ++kk) {
             const int c = kk >> 2, w = (kk & 3) * 32;
+            const int ch = kk % kSChains;
             const uint64_t ad = sdesc_kmajor_sw128(sbase + L::kQOff + c * (kRows * 128) + w);
             const uint64_t bd = sdesc_kmajor_sw128(kbase + c * (kBN * 128) + w);
-            umma_bf16(tmem + kSCol + sb * kBN, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+            umma_bf16(tmem + kSCol + (sb * kSChains + ch) * kBN, ad, bd, idesc_s,
+                      kk >= kSChains ? 1u : 0u);
           }
           umma_commit(s_full(sb));
         }
@@ -208,10 +214,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
       float s[kBN];
 #pragma unroll
       for (int h = 0; h < kBN / 32; ++h) {
-        tmem_ld32(lane_base + kSCol + sb * kBN + h * 32, v);
-        tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) s[h * 32 + e] = __uint_as_float(v[e]);
+        for (int ch = 0; ch < kSChains; ++ch) {   // chains summed in a fixed order
+          tmem_ld32(lane_base + kSCol + (sb * kSChains + ch) * kBN + h * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            s[h * 32 + e] = (ch == 0) ? __uint_as_float(v[e]) : s[h * 32 + e] + __uint_as_float(v[e]);
+        }
       }
       tc_fence_before();
       __syncwarp();

@@ -16,7 +16,7 @@ using namespace dg;
 
 namespace {
 
-constexpr int kGroupedTile = 128;   // B rows per grouped-GEMM tile
+constexpr int kGroupedTile = 64;    // B rows per grouped-GEMM tile (and per B box)
 constexpr int kMaxAttnChunks = 16;
 constexpr int kMaxSplits = 16;
 
@@ -44,6 +44,7 @@ struct dg_ctx {
   bool weights_ready = false;
 
   int Tmax = 0, NQKV = 0, G = 0;
+  int dense_box = 256;   // B rows per dense-GEMM tile: one TMA box covers all canvas rows
   bf16* embed = nullptr;
   float* ln_final = nullptr;
   std::vector<Layer> layers;
@@ -79,7 +80,7 @@ struct dg_ctx {
   int rope_P = -1;
   float* router_bias = nullptr;
   bool has_bias = false;
-  CUtensorMap m_x_b, m_x_a, m_attn_o_b, m_xperm_b, m_H_b;
+  CUtensorMap m_x_b, m_x_a, m_attn_o_b, m_xperm_b, m_H_b, m_x2_b;
   CUtensorMap m_q, m_kc, m_vc;   // attention operands
 
   int last_T = 0, last_B = 0, launches = 0;
@@ -220,10 +221,9 @@ int run_dense(dg_ctx* c, int kind, const CUtensorMap& mA, const CUtensorMap& mB,
   memset(&a, 0, sizeof(a));
   a.mode = GEMM_DENSE;
   a.M = M; a.N = N; a.K = K; a.n_kb = K / 64;
-  a.n_tile = std::min(256, (N + 31) / 32 * 32);
-  // wide activation tiles: pair two weight slabs per tile to halve B traffic
-  a.dense_pair = (a.n_tile >= 128 && M > 128) ? 1 : 0;
-  a.m_slabs = (M + 128 * (1 + a.dense_pair) - 1) / (128 * (1 + a.dense_pair));
+  a.n_tile = c->dense_box;      // one B box per stage covers the activation rows
+  a.b_box_rows = c->dense_box;
+  a.m_slabs = (M + 127) / 128;
   const int n_chunks = (N + a.n_tile - 1) / a.n_tile;
   a.k_splits = choose_splits(a.m_slabs * n_chunks, a.n_kb, c->num_sms);
   if ((size_t)a.k_splits * N * M > c->part_elems) a.k_splits = 1;
@@ -245,6 +245,7 @@ int run_grouped(dg_ctx* c, int mode, const CUtensorMap& mA, const CUtensorMap& m
   a.K = K; a.n_kb = K / 64;
   a.M = M;
   a.n_tile = kGroupedTile;
+  a.b_box_rows = kGroupedTile;
   a.m_slabs = (M + 127) / 128;
   a.n_groups = cf.n_experts + 1;
   a.offsets = c->offsets_g;
@@ -305,7 +306,7 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
                                 c->xperm, c->stream));
 
   // router
-  if ((rc = run_dense(c, K_GEMM_ROUTER, L.m_r, c->m_xperm_b, E, T, d, &splits)) != DG_OK) return rc;
+  if ((rc = run_dense(c, K_GEMM_ROUTER, L.m_r, c->m_x2_b, E, T, d, &splits)) != DG_OK) return rc;
   {
     RouterArgs ra;
     memset(&ra, 0, sizeof(ra));
@@ -481,6 +482,7 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
   const int d = cf.d_model, F = cf.d_ff, dh = cf.head_dim, E = cf.n_experts, k = cf.top_k;
   const int Hq = cf.n_q_heads, Hkv = cf.n_kv_heads;
   c->Tmax = cf.max_batch * cf.canvas_len;
+  c->dense_box = std::min(256, (c->Tmax + 31) / 32 * 32);
   c->NQKV = (Hq + 2 * Hkv) * dh;
   c->G = E + 1;
   const size_t T = c->Tmax, V = cf.vocab;
@@ -574,11 +576,12 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
     ok &= make_tmap_3d(&L.m_gu, L.wgu, d, 2 * F, c->G, 128);
     ok &= make_tmap_3d(&L.m_d, L.wd, F, d, c->G, 128);
   }
-  ok &= make_tmap_2d(&c->m_x_b, c->x, d, Tp, 32);
+  ok &= make_tmap_2d(&c->m_x_b, c->x, d, Tp, c->dense_box);
   ok &= make_tmap_2d(&c->m_x_a, c->x, d, Tp, 128);
-  ok &= make_tmap_2d(&c->m_attn_o_b, c->attn_o, (uint64_t)Hq * dh, Tp, 32);
-  ok &= make_tmap_2d(&c->m_xperm_b, c->xperm, d, rows_moe, 32);
-  ok &= make_tmap_2d(&c->m_H_b, c->H, F, rows_moe, 32);
+  ok &= make_tmap_2d(&c->m_attn_o_b, c->attn_o, (uint64_t)Hq * dh, Tp, c->dense_box);
+  ok &= make_tmap_2d(&c->m_xperm_b, c->xperm, d, rows_moe, kGroupedTile);
+  ok &= make_tmap_2d(&c->m_x2_b, c->xperm, d, rows_moe, c->dense_box);
+  ok &= make_tmap_2d(&c->m_H_b, c->H, F, rows_moe, kGroupedTile);
   ok &= make_tmap_2d(&c->m_q, c->q, dh, std::max<size_t>(T * Hq, 128), 128);
   ok &= make_tmap_2d(&c->m_kc, c->kc, dh, std::max<size_t>(T * Hkv, 64), 64);
   ok &= make_tmap_2d(&c->m_vc, c->vc, dh, std::max<size_t>(T * Hkv, 64), 64);

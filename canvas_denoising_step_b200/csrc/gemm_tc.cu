@@ -98,7 +98,7 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t) {
   // Tiles that run at the same time and share an operand (the slabs of one
   // projection or expert, the vocab blocks of the head) start their k loops at
   // different blocks so they do not all read the same lines at once.
-  ti.rot = ((a.mode == GEMM_HEAD ? ti.vb : ti.m_slab) * 5) % max(1, ti.kb1 - ti.kb0);
+  ti.rot = a.rotate ? ((a.mode == GEMM_HEAD ? ti.vb : ti.m_slab) * 5) % max(1, ti.kb1 - ti.kb0) : 0;
   if (a.mode == GEMM_HEAD) {
     ti.n_mma = 256;
     ti.n_bbox = 1;
@@ -157,7 +157,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   griddep_launch();
 
   const int n_tiles = tile_count(a);
-  const int n_bufs = (a.mode == GEMM_HEAD || (a.mode == GEMM_DENSE && a.dense_pair)) ? 1 : 2;
+  // TMEM layout: n_bufs tile buffers of 512/n_bufs columns; in a buffer,
+  // accumulator i, chain c starts at column (i * n_chain + c) * chain_cols.
+  const int n_bufs = a.n_bufs;
+  const uint32_t buf_cols = 512u / (uint32_t)n_bufs;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -211,7 +214,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         const uint32_t tph = (uint32_t)((it / n_bufs) & 1);
         if (!mbar_wait(tempty_bar(buf), tph ^ 1u, abort_flag, a.err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_base = tmem_base + (uint32_t)buf * 256u;
+        const uint32_t d_base = tmem_base + (uint32_t)buf * buf_cols;
         const uint32_t idesc = idesc_bf16_f32(ti.n_mma);
         const int nk = ti.kb1 - ti.kb0;
         for (int ik = 0; ik < nk; ++ik) {
@@ -221,11 +224,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
           const uint32_t sB = sA + (uint32_t)a.a_bytes;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
+            // consecutive k16 steps go to independent accumulator chains, so
+            // the tensor core is not held by one dependent accumulation
+            const int q = ik * (kBK / 16) + kk;
+            const int chain = q % a.n_chain;
             const uint64_t bdesc = sdesc_kmajor_sw128(sB + kk * 32);
             for (int i = 0; i < ti.n_acc; ++i) {
               const uint64_t adesc = sdesc_kmajor_sw128(sA + i * kATileBytes + kk * 32);
-              umma_bf16(d_base + (uint32_t)i * 256u, adesc, bdesc, idesc,
-                        (ik > 0 || kk > 0) ? 1u : 0u);
+              umma_bf16(d_base + (uint32_t)((i * a.n_chain + chain) * a.chain_cols), adesc, bdesc,
+                        idesc, q >= a.n_chain ? 1u : 0u);
             }
           }
           umma_commit(empty_bar(stage));
@@ -247,15 +254,26 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       const uint32_t tph = (uint32_t)((it / n_bufs) & 1);
       if (!mbar_wait(tfull_bar(buf), tph, abort_flag, a.err)) break;
       tc_fence_after();
-      const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)buf * 256u;
+      const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)buf * buf_cols;
       uint32_t v[32];
+      // columns c0 .. c0+31 of accumulator i, summed over the chains in order
+      auto load_acc = [&](int i, int c0) {
+        tmem_ld32(lane_addr + (uint32_t)(i * a.n_chain * a.chain_cols + c0), v);
+        tmem_wait_ld();
+        for (int c = 1; c < a.n_chain; ++c) {
+          uint32_t w[32];
+          tmem_ld32(lane_addr + (uint32_t)((i * a.n_chain + c) * a.chain_cols + c0), w);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(w[j]));
+        }
+      };
       if (a.mode == GEMM_DENSE || a.mode == GEMM_DOWN) {
         float* out = a.out_f32 + (size_t)ti.split * a.N * a.M;
         for (int i = 0; i < ti.n_acc; ++i) {
           const int m = ti.a_row0 + i * 128 + r;
           for (int c0 = 0; c0 < ti.n_mma; c0 += 32) {
-            tmem_ld32(lane_addr + (uint32_t)i * 256u + c0, v);
-            tmem_wait_ld();
+            load_acc(i, c0);
             if (m < a.M) {
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
@@ -271,8 +289,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         const int f = (ti.m_slab * 128 + r) >> 1;
         const bool is_gate = (r & 1) == 0;
         for (int c0 = 0; c0 < ti.n_mma; c0 += 32) {
-          tmem_ld32(lane_addr + c0, v);
-          tmem_wait_ld();
+          load_acc(0, c0);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float x = __uint_as_float(v[j]);
@@ -290,8 +307,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
           float mx = -INFINITY, sum = 0.f;
           int arg = -1;
           for (int c0 = 0; c0 < 256; c0 += 32) {
-            tmem_ld32(lane_addr + (uint32_t)i * 256u + c0, v);
-            tmem_wait_ld();
+            load_acc(i, c0);
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const int vid = ti.row0 + c0 + j;
@@ -380,16 +396,30 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t m
 }
 
 // Shared-memory plan: A region (1 or 2 tiles of 16 KB) + B region, as many
-// stages as fit in ~220 KB.
+// stages as fit in ~220 KB; and the TMEM plan: as many accumulator chains
+// (up to 4) as fit, preferring two tile buffers.
 void gemm_plan_smem(GemmArgs& a) {
+  {
+    const int n_acc = (a.mode == GEMM_HEAD || (a.mode == GEMM_DENSE && a.dense_pair)) ? 2 : 1;
+    const int n = (a.mode == GEMM_HEAD) ? 256 : a.n_tile;
+    a.chain_cols = ((n + 31) / 32) * 32;
+    int chains = 256 / (n_acc * a.chain_cols);
+    if (chains >= 2 || (chains >= 1 && a.mode != GEMM_DENSE)) {
+      a.n_bufs = 2;
+    } else {
+      a.n_bufs = 1;
+      chains = 512 / (n_acc * a.chain_cols);
+    }
+    a.n_chain = chains < 1 ? 1 : (chains > 4 ? 4 : chains);
+  }
   const int n_a = (a.mode == GEMM_HEAD || (a.mode == GEMM_DENSE && a.dense_pair)) ? 2 : 1;
   a.a_bytes = n_a * kATileBytes;
   if (a.mode == GEMM_HEAD) {
     a.b_box_rows = 256;
     a.b_bytes = 256 * 128;
   } else {
-    a.b_box_rows = 32;
-    a.b_bytes = ((a.n_tile + 31) / 32) * 32 * 128;
+    if (a.b_box_rows <= 0) a.b_box_rows = 32;   // must match the B tensor map's box
+    a.b_bytes = ((a.n_tile + a.b_box_rows - 1) / a.b_box_rows) * a.b_box_rows * 128;
   }
   a.stage_bytes = a.a_bytes + a.b_bytes;  // multiples of 1024
   int s = (220 * 1024) / a.stage_bytes;
