@@ -16,7 +16,8 @@ using namespace dg;
 
 namespace {
 
-constexpr int kGroupedTile = 64;    // B rows per grouped-GEMM tile (and per B box)
+constexpr int kGroupedTile = 128;   // B rows per grouped-GEMM tile
+constexpr int kGroupedBox = 32;     // B rows per TMA box of a grouped tile
 constexpr int kMaxAttnChunks = 16;
 constexpr int kMaxSplits = 16;
 
@@ -245,7 +246,7 @@ int run_grouped(dg_ctx* c, int mode, const CUtensorMap& mA, const CUtensorMap& m
   a.K = K; a.n_kb = K / 64;
   a.M = M;
   a.n_tile = kGroupedTile;
-  a.b_box_rows = kGroupedTile;
+  a.b_box_rows = kGroupedBox;
   a.m_slabs = (M + 127) / 128;
   a.n_groups = cf.n_experts + 1;
   a.offsets = c->offsets_g;
@@ -579,9 +580,9 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
   ok &= make_tmap_2d(&c->m_x_b, c->x, d, Tp, c->dense_box);
   ok &= make_tmap_2d(&c->m_x_a, c->x, d, Tp, 128);
   ok &= make_tmap_2d(&c->m_attn_o_b, c->attn_o, (uint64_t)Hq * dh, Tp, c->dense_box);
-  ok &= make_tmap_2d(&c->m_xperm_b, c->xperm, d, rows_moe, kGroupedTile);
+  ok &= make_tmap_2d(&c->m_xperm_b, c->xperm, d, rows_moe, kGroupedBox);
   ok &= make_tmap_2d(&c->m_x2_b, c->xperm, d, rows_moe, c->dense_box);
-  ok &= make_tmap_2d(&c->m_H_b, c->H, F, rows_moe, kGroupedTile);
+  ok &= make_tmap_2d(&c->m_H_b, c->H, F, rows_moe, kGroupedBox);
   ok &= make_tmap_2d(&c->m_q, c->q, dh, std::max<size_t>(T * Hq, 128), 128);
   ok &= make_tmap_2d(&c->m_kc, c->kc, dh, std::max<size_t>(T * Hkv, 64), 64);
   ok &= make_tmap_2d(&c->m_vc, c->vc, dh, std::max<size_t>(T * Hkv, 64), 64);

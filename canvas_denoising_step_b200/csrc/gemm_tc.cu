@@ -396,21 +396,18 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t m
 }
 
 // Shared-memory plan: A region (1 or 2 tiles of 16 KB) + B region, as many
-// stages as fit in ~220 KB; and the TMEM plan: as many accumulator chains
-// (up to 4) as fit, preferring two tile buffers.
+// stages as fit in ~220 KB; and the TMEM plan (tile buffers, accumulator
+// chains).
 void gemm_plan_smem(GemmArgs& a) {
   {
     const int n_acc = (a.mode == GEMM_HEAD || (a.mode == GEMM_DENSE && a.dense_pair)) ? 2 : 1;
     const int n = (a.mode == GEMM_HEAD) ? 256 : a.n_tile;
     a.chain_cols = ((n + 31) / 32) * 32;
-    int chains = 256 / (n_acc * a.chain_cols);
-    if (chains >= 2 || (chains >= 1 && a.mode != GEMM_DENSE)) {
-      a.n_bufs = 2;
-    } else {
-      a.n_bufs = 1;
-      chains = 512 / (n_acc * a.chain_cols);
-    }
-    a.n_chain = chains < 1 ? 1 : (chains > 4 ? 4 : chains);
+    // One chain: the GEMMs here are bound by how fast a CTA's shared memory
+    // fills, not by the MMA latency; extra chains measured slower for the
+    // small-N expert tiles and no faster for the dense ones.
+    a.n_chain = 1;
+    a.n_bufs = (n_acc * a.chain_cols <= 256) ? 2 : 1;
   }
   const int n_a = (a.mode == GEMM_HEAD || (a.mode == GEMM_DENSE && a.dense_pair)) ? 2 : 1;
   a.a_bytes = n_a * kATileBytes;
