@@ -4,7 +4,7 @@ Argument marshalling only: every function here forwards to the C function of
 the same name in ``libdg.so`` (declared in ``include/dg.h``).  Pointers are
 plain integers (``tensor.data_ptr()`` for torch tensors); torch is used by
 callers only for device memory and streams.  Importing fails loudly when the
-library has not been built (``python -m canvas_denoising_step_b200.build``).
+library has not been built (``python canvas_denoising_step_b200/build.py``).
 """
 
 from __future__ import annotations
@@ -51,7 +51,7 @@ class DgError(RuntimeError):
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
-                      "`python -m canvas_denoising_step_b200.build` (nvcc, sm_100a)")
+                      "`python canvas_denoising_step_b200/build.py` (nvcc, sm_100a)")
 
 _lib = ctypes.CDLL(LIB_PATH)
 

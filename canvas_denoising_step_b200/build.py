@@ -1,6 +1,7 @@
 """Builds libdg.so (the C-ABI canvas-step library) in-tree for sm_100a.
 
-    python -m canvas_denoising_step_b200.build          # or build() from Python
+    python canvas_denoising_step_b200/build.py     # or build() from Python (load this
+                                                   # file by path, not through the package)
 
 Each .cu under csrc/ is compiled with nvcc for sm_100a into _build/, then
 linked into canvas_denoising_step_b200/libdg.so (CUDA runtime linked

@@ -15,7 +15,7 @@ HEADER = os.path.join(ROOT, "include", "dg.h")
 
 @pytest.fixture(scope="module")
 def dg():
-    from canvas_denoising_step_b200.build import build
+    from libbuild import build_library as build
     build()
     import canvas_denoising_step_b200 as m
     return m

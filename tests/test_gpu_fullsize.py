@@ -20,7 +20,7 @@ pytestmark = pytest.mark.gpu
 def _cuda():
     if not torch.cuda.is_available():
         pytest.skip("needs a GPU")
-    from canvas_denoising_step_b200.build import build
+    from libbuild import build_library as build
     build()
     torch.cuda.set_device(0)
 

@@ -25,7 +25,7 @@ LAYER_TOL = 1e-2
 def _cuda():
     if not torch.cuda.is_available():
         pytest.skip("needs a GPU")
-    from canvas_denoising_step_b200.build import build
+    from libbuild import build_library as build
     build()
     torch.cuda.set_device(0)
 
