@@ -65,6 +65,8 @@ _SIGS = {
     "dg_denoise_block": (c_int, [c_void_p, c_void_p, c_int, c_int]),
     "dg_layer_forward": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_int]),
     "dg_router_topk": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "dg_router_topk_static": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
+                                      c_void_p, c_void_p, c_void_p]),
     "dg_commit": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p]),
     "dg_debug_tensor": (c_int, [c_void_p, c_char_p, c_void_p, c_size_t, POINTER(c_size_t)]),
     "dg_profile_enable": (c_int, [c_void_p, c_int]),
@@ -145,6 +147,15 @@ def dg_layer_forward(ctx: int, layer: int, x_in: int, x_out: int, n_rows: int) -
 def dg_router_topk(ctx: int, logits: int, n_rows: int, idx: int, w: int, offsets: int,
                    perm: int) -> None:
     _check(ctx, _lib.dg_router_topk(ctx, logits, n_rows, idx, w, offsets, perm), "dg_router_topk")
+
+
+def dg_router_topk_static(logits: int, n_rows: int, n_experts: int, top_k: int, idx: int, w: int,
+                          offsets: int, perm: int, stream: int = 0) -> None:
+    """Context-free router grouping that allocates no device memory (see dg.h)."""
+    code = _lib.dg_router_topk_static(logits, n_rows, n_experts, top_k, idx, w, offsets, perm,
+                                      stream)
+    if code != DG_OK:
+        raise DgError(code, "dg_router_topk_static", "rejected or failed")
 
 
 def dg_commit(ctx: int, conf: int, canvas: int, batch: int, steps_left: int, cand_tok: int,

@@ -157,6 +157,31 @@ int dg_layer_forward(dg_ctx* ctx, int layer, const void* x_in, void* x_out, int 
 int dg_router_topk(dg_ctx* ctx, const float* logits, int n_rows, int32_t* idx, float* w,
                    int32_t* offsets, int32_t* perm);
 
+/* dg_router_topk for callers that cannot allocate device memory.  The pages
+ * have no counterpart: this entry point exists for programs whose device
+ * memory is owned entirely by their own pool or arena, or that run under a
+ * rule forbidding allocation after start-up, and so cannot create a context
+ * (dg_create allocates weights and workspace) or let the library call
+ * cudaMalloc.  It takes no context and allocates nothing: the caller passes
+ * the inputs and outputs, exactly as for dg_router_topk (logits dev fp32
+ * [n_rows][n_experts], 16-byte aligned; idx, w, offsets, perm dev, same
+ * layouts), plus the expert count, top_k and a cudaStream_t (NULL = legacy
+ * default stream).  The scratch it needs (membership bitmap, last-block
+ * counter, inverse permutation: 131,328 bytes) is one fixed array in the
+ * library's device data, held by every GPU that loads the library until the
+ * process exits.  Limits: 1 <= n_rows <= 2048, n_experts a multiple of 4 in
+ * [4, 256], 1 <= top_k <= min(8, n_experts); larger sizes return
+ * DG_ERR_INVALID_ARG without touching the GPU.  The first call on a device
+ * looks up the array's device address (a runtime query, no allocation), so
+ * make that first call before any stream capture.  The scratch is cleared on
+ * the stream at the start of each call; calls share it, so calls that may
+ * overlap on the GPU (other streams, other host threads) race and must be
+ * serialised by the caller.  Returns DG_OK, DG_ERR_INVALID_ARG or
+ * DG_ERR_CUDA; the results are ready when the stream reaches them. */
+int dg_router_topk_static(const float* logits, int n_rows, int n_experts, int top_k,
+                          int32_t* idx, float* w, int32_t* offsets, int32_t* perm,
+                          void* cuda_stream);
+
 /* Commit test hook: the commit rule of dg_canvas_step on given confidences.
  * conf: dev fp32 [batch][canvas_len]; cand_tok: dev int32 [batch][canvas_len]
  * (the token each slot would receive); canvas: dev int32, in place;
