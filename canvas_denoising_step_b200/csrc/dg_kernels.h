@@ -13,7 +13,6 @@ struct GemmArgs {
   int n_tile;             // B rows per tile (DENSE / grouped)
   int k_splits;           // DENSE split-K
   int dense_pair;         // DENSE: tiles of two 128-row slabs (m_slabs counts pairs)
-  int rotate;             // start each tile's k loop at a tile-dependent block
   int m_slabs;            // 128-row slabs of A per group (DENSE / grouped)
   int n_groups;           // grouped: number of groups
   const int* offsets;     // grouped: [n_groups + 1] first B row of each group
@@ -29,7 +28,7 @@ struct GemmArgs {
   int* err;
   // shared-memory and TMEM plan (gemm_plan_smem)
   int stages, a_bytes, b_bytes, stage_bytes, b_box_rows;
-  int n_bufs, n_chain, chain_cols;
+  int n_bufs;
 };
 
 bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,

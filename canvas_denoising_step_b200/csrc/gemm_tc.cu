@@ -29,6 +29,7 @@ namespace {
 constexpr int kThreads = 192;
 constexpr int kBK = 64;             // K elements per stage (128-byte rows)
 constexpr int kATileBytes = 128 * 128;  // 128 rows x 128 B
+constexpr uint32_t kAccCols = 256;      // TMEM columns between the accumulators of a tile
 
 struct TileInfo {
   int g, m_slab, row0, rows, kb0, kb1, split, tb, vb;
@@ -36,7 +37,6 @@ struct TileInfo {
   int n_acc;   // accumulators (A tiles) per tile
   int n_mma;   // MMA N
   int n_bbox;  // B boxes per stage
-  int rot;     // the k-blocks run in the order kb0 + (rot + i) % (kb1 - kb0)
 };
 
 __device__ __forceinline__ int upper_bound_prefix(const int* prefix, int n, int c) {
@@ -95,10 +95,6 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t) {
     ti.kb1 = a.n_kb;
     ti.a_row0 = ti.tb * 256;
   }
-  // Tiles that run at the same time and share an operand (the slabs of one
-  // projection or expert, the vocab blocks of the head) start their k loops at
-  // different blocks so they do not all read the same lines at once.
-  ti.rot = a.rotate ? ((a.mode == GEMM_HEAD ? ti.vb : ti.m_slab) * 5) % max(1, ti.kb1 - ti.kb0) : 0;
   if (a.mode == GEMM_HEAD) {
     ti.n_mma = 256;
     ti.n_bbox = 1;
@@ -158,7 +154,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
 
   const int n_tiles = tile_count(a);
   // TMEM layout: n_bufs tile buffers of 512/n_bufs columns; in a buffer,
-  // accumulator i, chain c starts at column (i * n_chain + c) * chain_cols.
+  // accumulator i starts at column i * kAccCols.
   const int n_bufs = a.n_bufs;
   const uint32_t buf_cols = 512u / (uint32_t)n_bufs;
 
@@ -172,9 +168,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         const TileInfo ti = decode_tile(a, t);
         const uint32_t tx = (uint32_t)(ti.n_acc * kATileBytes) +
                             (uint32_t)(ti.n_bbox * a.b_box_rows * 128);
-        const int nk = ti.kb1 - ti.kb0;
-        for (int ik = 0; ik < nk; ++ik) {
-          const int kb = ti.kb0 + (ti.rot + ik) % nk;
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.err)) { ok = false; break; }
           const uint32_t sA = smem_base + (uint32_t)stage * a.stage_bytes;
           const uint32_t sB = sA + (uint32_t)a.a_bytes;
@@ -216,23 +210,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         tc_fence_after();
         const uint32_t d_base = tmem_base + (uint32_t)buf * buf_cols;
         const uint32_t idesc = idesc_bf16_f32(ti.n_mma);
-        const int nk = ti.kb1 - ti.kb0;
-        for (int ik = 0; ik < nk; ++ik) {
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sA = smem_base + (uint32_t)stage * a.stage_bytes;
           const uint32_t sB = sA + (uint32_t)a.a_bytes;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            // consecutive k16 steps go to independent accumulator chains, so
-            // the tensor core is not held by one dependent accumulation
-            const int q = ik * (kBK / 16) + kk;
-            const int chain = q % a.n_chain;
             const uint64_t bdesc = sdesc_kmajor_sw128(sB + kk * 32);
             for (int i = 0; i < ti.n_acc; ++i) {
               const uint64_t adesc = sdesc_kmajor_sw128(sA + i * kATileBytes + kk * 32);
-              umma_bf16(d_base + (uint32_t)((i * a.n_chain + chain) * a.chain_cols), adesc, bdesc,
-                        idesc, q >= a.n_chain ? 1u : 0u);
+              umma_bf16(d_base + (uint32_t)i * kAccCols, adesc, bdesc, idesc,
+                        (kb > ti.kb0 || kk > 0) ? 1u : 0u);
             }
           }
           umma_commit(empty_bar(stage));
@@ -256,24 +245,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       tc_fence_after();
       const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)buf * buf_cols;
       uint32_t v[32];
-      // columns c0 .. c0+31 of accumulator i, summed over the chains in order
-      auto load_acc = [&](int i, int c0) {
-        tmem_ld32(lane_addr + (uint32_t)(i * a.n_chain * a.chain_cols + c0), v);
-        tmem_wait_ld();
-        for (int c = 1; c < a.n_chain; ++c) {
-          uint32_t w[32];
-          tmem_ld32(lane_addr + (uint32_t)((i * a.n_chain + c) * a.chain_cols + c0), w);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(w[j]));
-        }
-      };
       if (a.mode == GEMM_DENSE || a.mode == GEMM_DOWN) {
         float* out = a.out_f32 + (size_t)ti.split * a.N * a.M;
         for (int i = 0; i < ti.n_acc; ++i) {
           const int m = ti.a_row0 + i * 128 + r;
           for (int c0 = 0; c0 < ti.n_mma; c0 += 32) {
-            load_acc(i, c0);
+            tmem_ld32(lane_addr + (uint32_t)i * kAccCols + (uint32_t)c0, v);
+            tmem_wait_ld();
             if (m < a.M) {
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
@@ -289,7 +267,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         const int f = (ti.m_slab * 128 + r) >> 1;
         const bool is_gate = (r & 1) == 0;
         for (int c0 = 0; c0 < ti.n_mma; c0 += 32) {
-          load_acc(0, c0);
+          tmem_ld32(lane_addr + (uint32_t)c0, v);
+          tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float x = __uint_as_float(v[j]);
@@ -307,7 +286,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
           float mx = -INFINITY, sum = 0.f;
           int arg = -1;
           for (int c0 = 0; c0 < 256; c0 += 32) {
-            load_acc(i, c0);
+            tmem_ld32(lane_addr + (uint32_t)i * kAccCols + (uint32_t)c0, v);
+            tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const int vid = ti.row0 + c0 + j;
@@ -396,20 +376,12 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t m
 }
 
 // Shared-memory plan: A region (1 or 2 tiles of 16 KB) + B region, as many
-// stages as fit in ~220 KB; and the TMEM plan (tile buffers, accumulator
-// chains).
+// stages as fit in ~220 KB; and the TMEM plan: two tile buffers of 256
+// columns when a tile has one accumulator (so the epilogue of one tile
+// overlaps the MMAs of the next), one buffer of two when it has two.
 void gemm_plan_smem(GemmArgs& a) {
-  {
-    const int n_acc = (a.mode == GEMM_HEAD || (a.mode == GEMM_DENSE && a.dense_pair)) ? 2 : 1;
-    const int n = (a.mode == GEMM_HEAD) ? 256 : a.n_tile;
-    a.chain_cols = ((n + 31) / 32) * 32;
-    // One chain: the GEMMs here are bound by how fast a CTA's shared memory
-    // fills, not by the MMA latency; extra chains measured slower for the
-    // small-N expert tiles and no faster for the dense ones.
-    a.n_chain = 1;
-    a.n_bufs = (n_acc * a.chain_cols <= 256) ? 2 : 1;
-  }
   const int n_a = (a.mode == GEMM_HEAD || (a.mode == GEMM_DENSE && a.dense_pair)) ? 2 : 1;
+  a.n_bufs = n_a == 1 ? 2 : 1;
   a.a_bytes = n_a * kATileBytes;
   if (a.mode == GEMM_HEAD) {
     a.b_box_rows = 256;
