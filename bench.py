@@ -129,9 +129,11 @@ def load_traffic(kernel):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms from before the
+    timed region to after it; only the samples stamped inside the region are kept
+    (the nearest later one when the region is shorter than the period)."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -140,6 +142,7 @@ class ClockSampler:
         ids = [v.strip() for v in vis.split(",") if v.strip()]
         self.gpu = ids[local_rank] if local_rank < len(ids) else str(local_rank)
         self.proc = None
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
@@ -149,25 +152,48 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+        time.sleep(0.5)    # nvidia-smi is sampling before the region opens
+
+    def mark_begin(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    @staticmethod
+    def _stamp(text):
+        import datetime
+        try:
+            return datetime.datetime.strptime(text.strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
 
     def stop(self):
         if not self.proc:
             return None
+        time.sleep(0.15)   # one more sample after the region closes
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 9]
         if not rows:
             return None
-        sm = [float(r[1]) for r in rows]
+        stamped = [(self._stamp(r[0]), r) for r in rows]
+        inside = [r for t, r in stamped if t is not None and self.t0 is not None and
+                  self.t0 <= t <= self.t1]
+        if not inside:
+            later = [r for t, r in stamped if t is not None and self.t0 is not None and t >= self.t0]
+            inside = later[:1] or rows[-1:]
+        sm = [float(r[2]) for r in inside]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Active" in v and
+        reasons = sorted({n for r in inside for n, v in zip(names, r[6:10]) if "Active" in v and
                           "Not" not in v})
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
-                "reasons": reasons, "samples": len(rows)}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(inside[0][3]),
+                "reasons": reasons, "samples": len(inside),
+                "power_w_median": statistics.median(float(r[4]) for r in inside)}
 
 
 # ----------------------------------------------------------------------------- CPU oracle timing
@@ -305,15 +331,17 @@ def run_ours(args, cfg, rank, world, local_rank):
         run_steps(args.warmup)
         dg.dg_sync(ctx)
         launches_per_step = dg.dg_last_launch_count(ctx)
-        barrier()
-        stream.synchronize()
         clocks = ClockSampler(local_rank)
         clocks.start()
+        barrier()
+        stream.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clocks.mark_begin()
         e0.record(stream)
         run_steps(args.steps)
         e1.record(stream)
         stream.synchronize()
+        clocks.mark_end()
         clk = clocks.stop()
         barrier()
         ms = e0.elapsed_time(e1)
@@ -455,7 +483,7 @@ def run_layer_case(args, cfg):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=32)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)

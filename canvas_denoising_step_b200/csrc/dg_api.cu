@@ -82,6 +82,7 @@ struct dg_ctx {
   float* router_bias = nullptr;
   bool has_bias = false;
   CUtensorMap m_x_b, m_x_a, m_attn_o_b, m_xperm_b, m_H_b, m_x2_b;
+  CUtensorMap m_Y_out;   // fp32 expert outputs [1][rows][d], tensor-store map
   CUtensorMap m_q, m_kc, m_vc;   // attention operands
 
   int last_T = 0, last_B = 0, launches = 0;
@@ -231,8 +232,12 @@ int run_dense(dg_ctx* c, int kind, const CUtensorMap& mA, const CUtensorMap& mB,
   a.out_f32 = c->part;
   a.err = c->err_dev;
   gemm_plan_smem(a);
+  // the split-K partials [k_splits][N][M], written by tensor stores
+  CUtensorMap mC;
+  if (!make_tmap_out_f32(&mC, c->part, (uint64_t)M, (uint64_t)N, (uint64_t)a.k_splits))
+    return fail(c, DG_ERR_CUDA, "tensor map for a projection output failed");
   const int tiles = a.m_slabs * n_chunks * a.k_splits;
-  DG_LAUNCH(c, kind, gemm_tc_launch(mA, mB, a, std::min(tiles, c->num_sms), c->stream));
+  DG_LAUNCH(c, kind, gemm_tc_launch(mA, mB, mC, a, std::min(tiles, c->num_sms), c->stream));
   *splits_out = a.k_splits;
   return DG_OK;
 }
@@ -258,7 +263,7 @@ int run_grouped(dg_ctx* c, int mode, const CUtensorMap& mA, const CUtensorMap& m
   (void)T;
   gemm_plan_smem(a);
   DG_LAUNCH(c, mode == GEMM_GATEUP ? K_GEMM_GATEUP : K_GEMM_DOWN,
-            gemm_tc_launch(mA, mB, a, c->num_sms, c->stream));
+            gemm_tc_launch(mA, mB, c->m_Y_out, a, c->num_sms, c->stream));
   return DG_OK;
 }
 
@@ -380,7 +385,8 @@ int record_step(dg_ctx* c, int B) {
   a.err = c->err_dev;
   gemm_plan_smem(a);
   const int tiles = a.n_vblocks * a.n_tblocks;
-  DG_LAUNCH(c, K_GEMM_HEAD, gemm_tc_launch(c->m_x_a, c->m_embed, a, std::min(tiles, c->num_sms), c->stream));
+  DG_LAUNCH(c, K_GEMM_HEAD, gemm_tc_launch(c->m_x_a, c->m_embed, c->m_Y_out, a,
+                                           std::min(tiles, c->num_sms), c->stream));
   DG_LAUNCH(c, K_HEAD_MERGE, launch_head_merge(c->head_m, c->head_s, c->head_a, a.n_vblocks, T, c->conf,
                                  c->tok, c->stream));
   DG_LAUNCH(c, K_COMMIT, launch_commit(c->conf, c->tok, c->canvas_dev, c->committed_dev, B, cf.canvas_len,
@@ -583,6 +589,7 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
   ok &= make_tmap_2d(&c->m_xperm_b, c->xperm, d, rows_moe, kGroupedBox);
   ok &= make_tmap_2d(&c->m_x2_b, c->xperm, d, rows_moe, c->dense_box);
   ok &= make_tmap_2d(&c->m_H_b, c->H, F, rows_moe, kGroupedBox);
+  ok &= make_tmap_out_f32(&c->m_Y_out, c->Y, d, rows_moe, 1);
   ok &= make_tmap_2d(&c->m_q, c->q, dh, std::max<size_t>(T * Hq, 128), 128);
   ok &= make_tmap_2d(&c->m_kc, c->kc, dh, std::max<size_t>(T * Hkv, 64), 64);
   ok &= make_tmap_2d(&c->m_vc, c->vc, dh, std::max<size_t>(T * Hkv, 64), 64);

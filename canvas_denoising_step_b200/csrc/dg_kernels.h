@@ -29,16 +29,24 @@ struct GemmArgs {
   // shared-memory and TMEM plan (gemm_plan_smem)
   int stages, a_bytes, b_bytes, stage_bytes, b_box_rows;
   int n_bufs;
+  int tab_bytes;          // group tables in shared memory (grouped modes)
+  int epi_bytes;          // fp32 output staging in shared memory (DENSE, DOWN)
 };
 
 bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                   uint32_t box_outer);
 bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid,
                   uint64_t outer, uint32_t box_mid);
+// fp32 [outer][mid][inner] output map for the DENSE / DOWN tensor stores.
+bool make_tmap_out_f32(CUtensorMap* map, float* base, uint64_t inner, uint64_t mid,
+                       uint64_t outer);
 void gemm_plan_smem(GemmArgs& a);
 size_t gemm_smem_bytes(const GemmArgs& a);
-cudaError_t gemm_tc_launch(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmArgs& a,
-                           int grid, cudaStream_t stream);
+// mapC: the fp32 output map (DENSE: [k_splits][N][M]; DOWN: [1][rows][M]); any
+// valid map for the other modes, which do not use it.
+cudaError_t gemm_tc_launch(const CUtensorMap& mapA, const CUtensorMap& mapB,
+                           const CUtensorMap& mapC, const GemmArgs& a, int grid,
+                           cudaStream_t stream);
 
 // ---------------------------------------------------------------- weight init
 // Physical layouts of the generated tensors (see init kernels).

@@ -5,6 +5,12 @@
 // (warp 1 also allocates TMEM); warps 2..5 are the epilogue, each reading its
 // 32-lane quadrant of TMEM with tcgen05.ld.  Accumulators are double
 // buffered so the epilogue of one tile overlaps the MMAs of the next.
+// The fp32 outputs (DENSE, DOWN) leave through shared memory: each epilogue
+// warp stages a 32 x 32 block and one lane writes it with a TMA tensor store
+// (blocks that end inside a group's rows, in DOWN, are written with masked
+// 16-byte stores instead, so that no row of the next group is touched).
+// The grouped modes copy the group tables (chunk prefix, row offsets) into
+// shared memory once, so tile decoding does not walk global memory.
 //
 // Operands are K-major bf16 tiles with the 128-byte swizzle (64 elements of
 // K per row).  The MMA is always M = 128: "A" rows are the output features
@@ -30,6 +36,7 @@ constexpr int kThreads = 192;
 constexpr int kBK = 64;             // K elements per stage (128-byte rows)
 constexpr int kATileBytes = 128 * 128;  // 128 rows x 128 B
 constexpr uint32_t kAccCols = 256;      // TMEM columns between the accumulators of a tile
+constexpr int kMaxSmem = 232448;        // dynamic shared memory per CTA (227 KB)
 
 struct TileInfo {
   int g, m_slab, row0, rows, kb0, kb1, split, tb, vb;
@@ -44,21 +51,23 @@ __device__ __forceinline__ int upper_bound_prefix(const int* prefix, int n, int 
   int lo = 0, hi = n;  // prefix[0] == 0 <= c
   while (hi - lo > 1) {
     int mid = (lo + hi) >> 1;
-    if (__ldg(prefix + mid) <= c) lo = mid; else hi = mid;
+    if (prefix[mid] <= c) lo = mid; else hi = mid;
   }
   return lo;
 }
 
-__device__ __forceinline__ int tile_count(const GemmArgs& a) {
+// s_prefix / s_offsets: the group tables in shared memory (grouped modes)
+__device__ __forceinline__ int tile_count(const GemmArgs& a, const int* s_prefix) {
   switch (a.mode) {
     case GEMM_DENSE: return a.m_slabs * ((a.N + a.n_tile - 1) / a.n_tile) * a.k_splits;
     case GEMM_GATEUP:
-    case GEMM_DOWN: return __ldg(a.chunk_prefix + a.n_groups) * a.m_slabs;
+    case GEMM_DOWN: return s_prefix[a.n_groups] * a.m_slabs;
     default: return a.n_vblocks * a.n_tblocks;
   }
 }
 
-__device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t) {
+__device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t, const int* s_prefix,
+                                               const int* s_offsets) {
   TileInfo ti;
   ti.g = 0; ti.split = 0; ti.tb = 0; ti.vb = 0; ti.n_acc = 1;
   if (a.mode == GEMM_DENSE) {
@@ -76,9 +85,9 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t) {
   } else if (a.mode == GEMM_GATEUP || a.mode == GEMM_DOWN) {
     ti.m_slab = t % a.m_slabs;
     const int c = t / a.m_slabs;
-    ti.g = upper_bound_prefix(a.chunk_prefix, a.n_groups, c);
-    const int j = c - __ldg(a.chunk_prefix + ti.g);
-    const int beg = __ldg(a.offsets + ti.g), end = __ldg(a.offsets + ti.g + 1);
+    ti.g = upper_bound_prefix(s_prefix, a.n_groups, c);
+    const int j = c - s_prefix[ti.g];
+    const int beg = s_offsets[ti.g], end = s_offsets[ti.g + 1];
     ti.row0 = beg + j * a.n_tile;
     ti.rows = min(a.n_tile, end - ti.row0);
     ti.kb0 = 0;
@@ -109,7 +118,7 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t) {
 
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-               const GemmArgs a) {
+               const __grid_constant__ CUtensorMap mapC, const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -152,7 +161,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   griddep_wait();
   griddep_launch();
 
-  const int n_tiles = tile_count(a);
+  // group tables (written by the router, the kernel before) into shared memory
+  int* s_prefix = reinterpret_cast<int*>(smem + (size_t)S * a.stage_bytes + 1024);
+  int* s_offsets = s_prefix + (a.n_groups + 1);
+  float* s_stage_out = reinterpret_cast<float*>(smem + (size_t)S * a.stage_bytes + 1024 + a.tab_bytes);
+  if (a.mode == GEMM_GATEUP || a.mode == GEMM_DOWN) {
+    for (int i = threadIdx.x; i <= a.n_groups; i += blockDim.x) {
+      s_prefix[i] = __ldg(a.chunk_prefix + i);
+      s_offsets[i] = __ldg(a.offsets + i);
+    }
+    __syncthreads();
+  }
+
+  const int n_tiles = tile_count(a, s_prefix);
   // TMEM layout: n_bufs tile buffers of 512/n_bufs columns; in a buffer,
   // accumulator i starts at column i * kAccCols.
   const int n_bufs = a.n_bufs;
@@ -165,7 +186,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       uint32_t phase = 0;
       bool wrapped = false, ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        const TileInfo ti = decode_tile(a, t);
+        const TileInfo ti = decode_tile(a, t, s_prefix, s_offsets);
         const uint32_t tx = (uint32_t)(ti.n_acc * kATileBytes) +
                             (uint32_t)(ti.n_bbox * a.b_box_rows * 128);
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
@@ -203,7 +224,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       bool ok = true;
       int it = 0;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
-        const TileInfo ti = decode_tile(a, t);
+        const TileInfo ti = decode_tile(a, t, s_prefix, s_offsets);
         const int buf = it % n_bufs;
         const uint32_t tph = (uint32_t)((it / n_bufs) & 1);
         if (!mbar_wait(tempty_bar(buf), tph ^ 1u, abort_flag, a.err)) { ok = false; break; }
@@ -236,9 +257,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;                 // TMEM lane quadrant of this warp
     const int r = q * 32 + lane;            // accumulator row (TMEM lane)
+    // staging blocks of this warp for the fp32 outputs: n_sbuf of 32 x 32 fp32
+    const int n_sbuf = a.epi_bytes / (4 * 4096);
+    float* s_warp_out = s_stage_out + (warp - 2) * n_sbuf * 1024;
+    int sbuf = 0;
     int it = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
-      const TileInfo ti = decode_tile(a, t);
+      const TileInfo ti = decode_tile(a, t, s_prefix, s_offsets);
       const int buf = it % n_bufs;
       const uint32_t tph = (uint32_t)((it / n_bufs) & 1);
       if (!mbar_wait(tfull_bar(buf), tph, abort_flag, a.err)) break;
@@ -246,18 +271,43 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)buf * buf_cols;
       uint32_t v[32];
       if (a.mode == GEMM_DENSE || a.mode == GEMM_DOWN) {
+        // out[split][row][m]; this warp holds rows m0 .. m0+31 of the tile
         float* out = a.out_f32 + (size_t)ti.split * a.N * a.M;
         for (int i = 0; i < ti.n_acc; ++i) {
-          const int m = ti.a_row0 + i * 128 + r;
+          const int m0 = ti.a_row0 + i * 128 + q * 32;
           for (int c0 = 0; c0 < ti.n_mma; c0 += 32) {
             tmem_ld32(lane_addr + (uint32_t)i * kAccCols + (uint32_t)c0, v);
             tmem_wait_ld();
-            if (m < a.M) {
+            float* st = s_warp_out + sbuf * 1024;   // [32 rows n][32 m]
+            // the store that last read this block has finished reading it
+            if (lane == 0) {
+              if (n_sbuf > 1) bulk_wait_read<1>(); else bulk_wait_read<0>();
+            }
+            __syncwarp();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int n = c0 + j;
-                if (n < ti.rows) out[(size_t)(ti.row0 + n) * a.M + m] = __uint_as_float(v[j]);
+            for (int j = 0; j < 32; ++j) st[j * 32 + lane] = __uint_as_float(v[j]);
+            if (a.mode == GEMM_DENSE || c0 + 32 <= ti.rows) {
+              // rows past N (DENSE) and m past M are clipped by the tensor map;
+              // a block with nothing inside is not stored at all
+              if (m0 < a.M) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                  tma_store_3d(&mapC, smem_u32(st), m0, ti.row0 + c0, ti.split);
+                  bulk_commit();
+                }
+                sbuf = (sbuf + 1 == n_sbuf) ? 0 : sbuf + 1;
               }
+            } else {
+              __syncwarp();
+#pragma unroll
+              for (int it2 = 0; it2 < 8; ++it2) {
+                const int nl = it2 * 4 + (lane >> 3), mo = 4 * (lane & 7);
+                if (c0 + nl < ti.rows && m0 + mo < a.M)
+                  *reinterpret_cast<float4*>(out + (size_t)(ti.row0 + c0 + nl) * a.M + m0 + mo) =
+                      *reinterpret_cast<const float4*>(st + nl * 32 + mo);
+              }
+              __syncwarp();
             }
           }
         }
@@ -315,6 +365,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty_bar(buf));
     }
+    // tensor stores of this warp complete before the CTA exits
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -375,13 +428,34 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t m
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 output [outer][mid][inner] written in 32 x 32 blocks (no swizzle):
+// elements past any extent are not written by a tensor store.
+bool make_tmap_out_f32(CUtensorMap* map, float* base, uint64_t inner, uint64_t mid,
+                       uint64_t outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, mid, outer};
+  cuuint64_t strides[2] = {inner * 4, inner * mid * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Shared-memory plan: A region (1 or 2 tiles of 16 KB) + B region, as many
-// stages as fit in ~220 KB; and the TMEM plan: two tile buffers of 256
+// stages as fit beside the barriers, group tables and output staging; and the
+// TMEM plan: two tile buffers of 256
 // columns when a tile has one accumulator (so the epilogue of one tile
 // overlaps the MMAs of the next), one buffer of two when it has two.
 void gemm_plan_smem(GemmArgs& a) {
   const int n_a = (a.mode == GEMM_HEAD || (a.mode == GEMM_DENSE && a.dense_pair)) ? 2 : 1;
   a.n_bufs = n_a == 1 ? 2 : 1;
+  // group tables; fp32 output staging: two 4 KB blocks per epilogue warp for
+  // DENSE, one for DOWN (which keeps its sixth operand stage)
+  a.tab_bytes = (a.mode == GEMM_GATEUP || a.mode == GEMM_DOWN)
+                    ? ((2 * (a.n_groups + 1) * 4 + 127) / 128) * 128 : 0;
+  a.epi_bytes = a.mode == GEMM_DENSE ? 2 * 4 * 4096 : (a.mode == GEMM_DOWN ? 4 * 4096 : 0);
   a.a_bytes = n_a * kATileBytes;
   if (a.mode == GEMM_HEAD) {
     a.b_box_rows = 256;
@@ -391,25 +465,28 @@ void gemm_plan_smem(GemmArgs& a) {
     a.b_bytes = ((a.n_tile + a.b_box_rows - 1) / a.b_box_rows) * a.b_box_rows * 128;
   }
   a.stage_bytes = a.a_bytes + a.b_bytes;  // multiples of 1024
-  int s = (220 * 1024) / a.stage_bytes;
+  int s = (int)((kMaxSmem - 2048 - a.tab_bytes - a.epi_bytes) / a.stage_bytes);
   a.stages = s < 2 ? 2 : (s > 8 ? 8 : s);
 }
 
 size_t gemm_smem_bytes(const GemmArgs& a) {
-  return 1024 + (size_t)a.stages * a.stage_bytes + (2 * a.stages + 4) * 8 + 16;
+  // alignment slack, stages, barriers (1 KB), group tables, output staging
+  return 1024 + (size_t)a.stages * a.stage_bytes + 1024 + a.tab_bytes + a.epi_bytes;
 }
 
-cudaError_t gemm_tc_launch(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmArgs& a,
-                           int grid, cudaStream_t stream) {
+cudaError_t gemm_tc_launch(const CUtensorMap& mapA, const CUtensorMap& mapB,
+                           const CUtensorMap& mapC, const GemmArgs& a, int grid,
+                           cudaStream_t stream) {
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
+  if (gemm_smem_bytes(a) > (size_t)kMaxSmem) return cudaErrorInvalidValue;
   return launch_k(gemm_tc_kernel, dim3(grid), dim3(kThreads), gemm_smem_bytes(a), stream, mapA,
-                  mapB, a);
+                  mapB, mapC, a);
 }
 
 }  // namespace dg
