@@ -157,7 +157,30 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // everything above overlaps the previous kernel's tail; data access starts here
+  // Everything above overlaps the previous kernel's tail.  The weights do not
+  // depend on it: in DENSE and HEAD the producer issues the weight operand of
+  // its first tile's first stages now (fresh barriers, no empty waits), and
+  // only the activation operand after the wait below.
+  int pre = 0;
+  if (warp == 0 && lane == 0 && (a.mode == GEMM_DENSE || a.mode == GEMM_HEAD) &&
+      (int)blockIdx.x < tile_count(a, nullptr)) {
+    const TileInfo ti = decode_tile(a, blockIdx.x, nullptr, nullptr);
+    const uint32_t tx = (uint32_t)(ti.n_acc * kATileBytes) +
+                        (uint32_t)(ti.n_bbox * a.b_box_rows * 128);
+    pre = min(S, ti.kb1 - ti.kb0);
+    for (int p = 0; p < pre; ++p) {
+      const uint32_t sA = smem_base + (uint32_t)p * a.stage_bytes;
+      const int kx = (ti.kb0 + p) * kBK;
+      mbar_arrive_expect_tx(full_bar(p), tx);
+      if (a.mode == GEMM_DENSE) {
+        for (int i = 0; i < ti.n_acc; ++i)
+          tma_load_2d(sA + i * kATileBytes, &mapA, full_bar(p), kx, ti.a_row0 + i * 128);
+      } else {
+        tma_load_2d(sA + (uint32_t)a.a_bytes, &mapB, full_bar(p), kx, ti.row0);
+      }
+    }
+  }
+  // data written by the previous kernel is read from here on
   griddep_wait();
   griddep_launch();
 
@@ -185,26 +208,36 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       int stage = 0;
       uint32_t phase = 0;
       bool wrapped = false, ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      bool first = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, first = false) {
         const TileInfo ti = decode_tile(a, t, s_prefix, s_offsets);
         const uint32_t tx = (uint32_t)(ti.n_acc * kATileBytes) +
                             (uint32_t)(ti.n_bbox * a.b_box_rows * 128);
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.err)) { ok = false; break; }
+          // the weight operand of this stage went out before the grid wait
+          const bool weight_issued = first && kb - ti.kb0 < pre;
           const uint32_t sA = smem_base + (uint32_t)stage * a.stage_bytes;
           const uint32_t sB = sA + (uint32_t)a.a_bytes;
           const uint32_t fb = full_bar(stage);
-          mbar_arrive_expect_tx(fb, tx);
           const int kx = kb * kBK;
-          if (a.mode == GEMM_DENSE || a.mode == GEMM_HEAD) {
+          if (!weight_issued) {
+            if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.err)) { ok = false; break; }
+            mbar_arrive_expect_tx(fb, tx);
+          }
+          if (a.mode == GEMM_DENSE) {
+            if (!weight_issued)
+              for (int i = 0; i < ti.n_acc; ++i)
+                tma_load_2d(sA + i * kATileBytes, &mapA, fb, kx, ti.a_row0 + i * 128);
+          } else if (a.mode == GEMM_HEAD) {
             for (int i = 0; i < ti.n_acc; ++i)
               tma_load_2d(sA + i * kATileBytes, &mapA, fb, kx, ti.a_row0 + i * 128);
           } else {
             tma_load_3d(sA, &mapA, fb, kx, ti.a_row0, ti.g);
           }
-          for (int i = 0; i < ti.n_bbox; ++i)
-            tma_load_2d(sB + (uint32_t)(i * a.b_box_rows * 128), &mapB, fb, kx,
-                        ti.row0 + i * a.b_box_rows);
+          if (!(weight_issued && a.mode == GEMM_HEAD))
+            for (int i = 0; i < ti.n_bbox; ++i)
+              tma_load_2d(sB + (uint32_t)(i * a.b_box_rows * 128), &mapB, fb, kx,
+                          ti.row0 + i * a.b_box_rows);
           if (++stage == S) { stage = 0; phase ^= 1u; wrapped = true; }
         }
       }

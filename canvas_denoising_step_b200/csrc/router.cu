@@ -34,10 +34,10 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
     float v[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = 0.f;
-    for (int s0 = 0; s0 < a.splits; s0 += 4) {
-      float4 buf[4][2];
+    for (int s0 = 0; s0 < a.splits; s0 += 8) {   // 8 splits' loads in flight at once
+      float4 buf[8][2];
 #pragma unroll
-      for (int ss = 0; ss < 4; ++ss)
+      for (int ss = 0; ss < 8; ++ss)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int e0 = 128 * hh + 4 * lane;
@@ -46,7 +46,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
                 a.logits_in + ((size_t)(s0 + ss) * T + t) * E + e0));
         }
 #pragma unroll
-      for (int ss = 0; ss < 4; ++ss)
+      for (int ss = 0; ss < 8; ++ss)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int e0 = 128 * hh + 4 * lane;
@@ -134,26 +134,53 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
     count[e] = run;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    int crun = a.n_shared ? (T + a.n_tile - 1) / a.n_tile : 0;
-    if (a.offsets_g) a.offsets_g[0] = 0;
-    if (a.chunk_prefix) { a.chunk_prefix[0] = 0; a.chunk_prefix[1] = crun; }
-    int active = 0;
-    for (int e = 0; e < E; ++e) {
-      off[e] = run;
-      if (a.offsets_r) a.offsets_r[e] = run;
-      if (a.offsets_g) a.offsets_g[e + 1] = T + run;
-      run += count[e];
-      active += count[e] > 0;
-      crun += (count[e] + a.n_tile - 1) / a.n_tile;
-      if (a.chunk_prefix) a.chunk_prefix[e + 2] = crun;
+  if (warp == 0) {
+    // offsets and chunk counts: an exclusive scan over the experts, lane l
+    // taking the `per` consecutive experts from l * per (integer arithmetic,
+    // so the result equals the sequential scan)
+    const int per = (E + 31) / 32;
+    const int base_chunks = a.n_shared ? (T + a.n_tile - 1) / a.n_tile : 0;
+    int c_cnt = 0, c_chk = 0, c_act = 0;
+    for (int q = 0; q < per; ++q) {
+      const int e = lane * per + q;
+      if (e < E) {
+        c_cnt += count[e];
+        c_chk += (count[e] + a.n_tile - 1) / a.n_tile;
+        c_act += count[e] > 0;
+      }
     }
-    off[E] = run;
-    if (a.offsets_r) a.offsets_r[E] = run;
-    if (a.offsets_g) a.offsets_g[E + 1] = T + run;
-    if (a.active_out) atomicAdd(a.active_out, active);
-    if (run != T * k) raise_error(a.err, kErrFault);
+    int s_cnt = c_cnt, s_chk = c_chk;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int vc = __shfl_up_sync(0xffffffffu, s_cnt, o);
+      const int vk = __shfl_up_sync(0xffffffffu, s_chk, o);
+      if (lane >= o) { s_cnt += vc; s_chk += vk; }
+    }
+    int run = s_cnt - c_cnt;
+    int crun = base_chunks + s_chk - c_chk;
+    for (int q = 0; q < per; ++q) {
+      const int e = lane * per + q;
+      if (e < E) {
+        off[e] = run;
+        if (a.offsets_r) a.offsets_r[e] = run;
+        if (a.offsets_g) a.offsets_g[e + 1] = T + run;
+        run += count[e];
+        crun += (count[e] + a.n_tile - 1) / a.n_tile;
+        if (a.chunk_prefix) a.chunk_prefix[e + 2] = crun;
+      }
+    }
+    const int total = __shfl_sync(0xffffffffu, s_cnt, 31);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c_act += __shfl_xor_sync(0xffffffffu, c_act, o);
+    if (lane == 0) {
+      if (a.offsets_g) a.offsets_g[0] = 0;
+      if (a.chunk_prefix) { a.chunk_prefix[0] = 0; a.chunk_prefix[1] = base_chunks; }
+      off[E] = total;
+      if (a.offsets_r) a.offsets_r[E] = total;
+      if (a.offsets_g) a.offsets_g[E + 1] = T + total;
+      if (a.active_out) atomicAdd(a.active_out, c_act);
+      if (total != T * k) raise_error(a.err, kErrFault);
+    }
   }
   __syncthreads();
   for (int i0 = 0; i0 < T * k; i0 += 8 * kRouterThreads) {  // 8 index loads in flight per thread
