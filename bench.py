@@ -110,9 +110,15 @@ def load_peaks():
 
 
 def kernel_src_sha():
+    """Hash of what the GEMM kernel is built from: gemm_tc.cu, dg_common.cuh and
+    the GemmArgs declaration (other declarations in dg_kernels.h do not count)."""
+    csrc = os.path.join(ROOT, "canvas_denoising_step_b200", "csrc")
     h = hashlib.sha256()
-    for f in ("gemm_tc.cu", "dg_common.cuh", "dg_kernels.h"):
-        h.update(open(os.path.join(ROOT, "canvas_denoising_step_b200", "csrc", f), "rb").read())
+    for f in ("gemm_tc.cu", "dg_common.cuh"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    hdr = open(os.path.join(csrc, "dg_kernels.h"), "rb").read()
+    i = hdr.index(b"struct GemmArgs")
+    h.update(hdr[i:hdr.index(b"};", i)])
     return h.hexdigest()[:16]
 
 

@@ -91,6 +91,7 @@ cudaError_t launch_qkv_rope(const float* part, int splits, int T, int Tc, int Hq
                             int n_rot, const float* cos_t, const float* sin_t, bf16* q, bf16* kc,
                             bf16* vc, cudaStream_t s);
 
+// Shape of the split-KV attention partials (read by the merge).
 struct AttnArgs {
   const bf16* q;   // [B][Hq][Tc][dh]
   const bf16* kc;  // [B][Hkv][Tc][dh]
@@ -104,9 +105,10 @@ struct AttnArgs {
   float* part_ml;  // [n_chunks][B*Hq*Tc][2]  (max in log2 units, sum)
   float scale_log2;  // log2(e) / sqrt(dh)
 };
-cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
 
-// tcgen05 attention (attention_tc.cu): same partial outputs as launch_attention.
+// tcgen05 attention (attention_tc.cu): writes the split-KV partials part_o /
+// part_ml in the AttnArgs layout above; launch_attn_merge (attn_merge.cu)
+// combines them.
 struct AttnTcArgs {
   int B, Hq, Hkv, Tc, P, dh;
   int n_vis;
