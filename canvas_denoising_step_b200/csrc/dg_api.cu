@@ -65,6 +65,8 @@ struct dg_ctx {
   float* w = nullptr;
   uint32_t* bitmap = nullptr;
   int* router_counter = nullptr;
+  int* chunk_ready = nullptr;        // per-chunk gate/up -> down hand-over counters
+  int n_chunk_ready = 0;
   int32_t *offsets_r = nullptr, *offsets_g = nullptr, *chunk_prefix = nullptr;
   int32_t *perm = nullptr, *inv = nullptr;
   bf16* H = nullptr;
@@ -260,6 +262,9 @@ int run_grouped(dg_ctx* c, int mode, const CUtensorMap& mA, const CUtensorMap& m
   a.out_f32 = c->Y;
   a.out_bf16 = c->H;
   a.err = c->err_dev;
+  // gate/up hands each chunk's H rows to down as soon as its slabs are written
+  a.chunk_ready = c->chunk_ready;
+  a.ready_target = 4 * ((2 * cf.d_ff + 127) / 128);   // epilogue warps x gate/up slabs
   (void)T;
   gemm_plan_smem(a);
   DG_LAUNCH(c, mode == GEMM_GATEUP ? K_GEMM_GATEUP : K_GEMM_DOWN,
@@ -322,6 +327,7 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
     ra.logits_out = c->router_logits; ra.idx = c->idx; ra.w = c->w;
     ra.bitmap = c->bitmap; ra.counter = c->router_counter;
     ra.offsets_r = c->offsets_r; ra.offsets_g = c->offsets_g; ra.chunk_prefix = c->chunk_prefix;
+    ra.chunk_ready = c->chunk_ready; ra.n_chunk_ready = c->n_chunk_ready;
     ra.perm = c->perm; ra.inv = c->inv; ra.active_out = c->expert_active + l; ra.err = c->err_dev;
     DG_LAUNCH(c, K_ROUTER, launch_router(ra, c->stream));
   }
@@ -530,6 +536,10 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
     ok &= alloc_n(c, &c->w, T * k);
     ok &= alloc_n(c, &c->bitmap, (size_t)E * ((T + 31) / 32));
     ok &= alloc_n(c, &c->router_counter, 4);
+    // every expert chunk of a layer: the shared group's plus the routed groups'
+    c->n_chunk_ready = (int)((T + kGroupedTile - 1) / kGroupedTile +
+                             ((size_t)k * T + kGroupedTile - 1) / kGroupedTile + E);
+    ok &= alloc_n(c, &c->chunk_ready, (size_t)c->n_chunk_ready);
     ok &= alloc_n(c, &c->steps_dev, 4);
     ok &= alloc_n(c, &c->offsets_r, E + 1);
     ok &= alloc_n(c, &c->offsets_g, E + 2);
@@ -563,6 +573,7 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
   // zero the scratch that kernels accumulate into or read before writing
   cudaMemset(c->bitmap, 0, (size_t)E * ((T + 31) / 32) * 4);
   cudaMemset(c->router_counter, 0, 16);
+  cudaMemset(c->chunk_ready, 0, sizeof(int) * (size_t)c->n_chunk_ready);
   cudaMemset(c->err_dev, 0, 16);
   cudaMemset(c->expert_active, 0, sizeof(int) * cf.n_layers);
   cudaMemset(c->xperm, 0, rows_moe * d * 2);

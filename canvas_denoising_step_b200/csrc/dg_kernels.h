@@ -29,6 +29,12 @@ struct GemmArgs {
   // shared-memory and TMEM plan (gemm_plan_smem)
   int stages, a_bytes, b_bytes, stage_bytes, b_box_rows;
   int n_bufs;
+  // Gate/up -> down hand-over without a whole-grid wait: GATEUP adds 1 to
+  // chunk_ready[c] per epilogue warp once its H rows of chunk c are written;
+  // DOWN (which then skips the grid dependency wait) loads a chunk's H rows
+  // once chunk_ready[c] reaches ready_target.  NULL: not used.
+  int* chunk_ready;
+  int ready_target;
   int tab_bytes;          // group tables in shared memory (grouped modes)
   int epi_bytes;          // fp32 output staging in shared memory (DENSE, DOWN)
 };
@@ -157,6 +163,8 @@ struct RouterArgs {
   int32_t* perm;           // [T*k]
   int32_t* inv;            // [T*k]
   int* active_out;         // += experts given rows, or NULL
+  int* chunk_ready;        // [n_chunk_ready] set to 0 (the expert GEMMs' counters), or NULL
+  int n_chunk_ready;
   int* err;
 };
 size_t router_smem_bytes(int T, int E);

@@ -114,6 +114,15 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t, const 
   return ti;
 }
 
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// the chunk index of a grouped tile (the same numbering in GATEUP and DOWN)
+__device__ __forceinline__ int tile_chunk(const GemmArgs& a, int t) { return t / a.m_slabs; }
+
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -180,8 +189,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       }
     }
   }
-  // data written by the previous kernel is read from here on
-  griddep_wait();
+  // Data written by the previous kernel is read from here on.  A DOWN launch
+  // with ready counters does not wait for the whole gate/up grid: its H rows
+  // are guarded per chunk below, and what else it reads (the group tables)
+  // was complete before the gate/up grid let it launch.
+  const bool handover = a.mode == GEMM_DOWN && a.chunk_ready != nullptr;
+  if (!handover) griddep_wait();
   griddep_launch();
 
   // group tables (written by the router, the kernel before) into shared memory
@@ -190,8 +203,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   float* s_stage_out = reinterpret_cast<float*>(smem + (size_t)S * a.stage_bytes + 1024 + a.tab_bytes);
   if (a.mode == GEMM_GATEUP || a.mode == GEMM_DOWN) {
     for (int i = threadIdx.x; i <= a.n_groups; i += blockDim.x) {
-      s_prefix[i] = __ldg(a.chunk_prefix + i);
-      s_offsets[i] = __ldg(a.offsets + i);
+      s_prefix[i] = __ldcg(a.chunk_prefix + i);
+      s_offsets[i] = __ldcg(a.offsets + i);
     }
     __syncthreads();
   }
@@ -213,6 +226,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         const TileInfo ti = decode_tile(a, t, s_prefix, s_offsets);
         const uint32_t tx = (uint32_t)(ti.n_acc * kATileBytes) +
                             (uint32_t)(ti.n_bbox * a.b_box_rows * 128);
+        if (handover) {
+          // this chunk's H rows are written by every gate/up slab's epilogue
+          const int* rc = a.chunk_ready + tile_chunk(a, t);
+          const unsigned long long t0 = globaltimer_ns();
+          while (ld_acquire(rc) < a.ready_target) {
+            if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
+              *abort_flag = 1;
+              raise_error(a.err, kErrTimeout);
+              ok = false;
+              break;
+            }
+          }
+          if (!ok) break;
+          fence_proxy_async_global();   // the TMA loads below see those writes
+        }
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           // the weight operand of this stage went out before the grid wait
           const bool weight_issued = first && kb - ti.kb0 < pre;
@@ -362,6 +390,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
               a.out_bf16[(size_t)(ti.row0 + n) * a.F + f] = f_to_bf16(h);
             }
           }
+        }
+        if (a.chunk_ready) {
+          // this warp's H writes of the tile are visible before the count
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) atomicAdd(a.chunk_ready + tile_chunk(a, t), 1);
         }
       } else {  // HEAD
         for (int i = 0; i < ti.n_acc; ++i) {

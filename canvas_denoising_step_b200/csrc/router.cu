@@ -204,6 +204,9 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
   }
   __syncthreads();
   for (int i = threadIdx.x; i < E * W; i += blockDim.x) a.bitmap[i] = 0u;
+  // the expert GEMMs' per-chunk ready counters start this layer at zero
+  if (a.chunk_ready)
+    for (int i = threadIdx.x; i < a.n_chunk_ready; i += blockDim.x) a.chunk_ready[i] = 0;
   if (threadIdx.x == 0) *a.counter = 0;
 }
 
