@@ -116,6 +116,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The prompt K/V is set before the pass and never written by it: the
+  // producer issues the first ring stages of prompt blocks before the grid
+  // wait (fresh barriers, no empty waits); q and the canvas K/V come after it.
+  auto issue_kv = [&](int j) {
+    const int st = j % kStages;
+    const int jg = jb0 + j;
+    const CUtensorMap* mk;
+    const CUtensorMap* mv;
+    int row;
+    if (jg < nbp) {
+      mk = &mapKp; mv = &mapVp;
+      row = (b * a.Hkv + g) * a.P + (a.P - a.n_vis) + jg * kBN;
+    } else {
+      mk = &mapKc; mv = &mapVc;
+      row = (b * a.Hkv + g) * a.Tc + (jg - nbp) * kBN;
+    }
+    mbar_arrive_expect_tx(kv_full(st), (uint32_t)(2 * L::kKV));
+    for (int c = 0; c < DH / 64; ++c) {
+      tma_load_2d(sbase + L::kKOff + st * L::kKV + c * (kBN * 128), mk, kv_full(st), c * 64, row);
+      tma_load_2d(sbase + L::kVOff + st * L::kKV + c * (kBN * 128), mv, kv_full(st), c * 64, row);
+    }
+  };
+  int pre_kv = 0;
+  if (warp == 0 && lane == 0)
+    while (pre_kv < kStages && pre_kv < n_local && jb0 + pre_kv < nbp) issue_kv(pre_kv++);
   griddep_wait();
   griddep_launch();
 
@@ -127,27 +152,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
       for (int c = 0; c < DH / 64; ++c)
         tma_load_2d(sbase + L::kQOff + c * (kRows * 128), &mapQ, q_full, c * 64, q_row0);
       bool ok = true;
-      int issued = 0;
-      for (int j = 0; j < n_local && ok; ++j) {
+      int issued = pre_kv;
+      for (int j = pre_kv; j < n_local && ok; ++j) {
         const int st = j % kStages;
         const uint32_t par = (uint32_t)((j / kStages) & 1) ^ 1u;
         if (!mbar_wait(kv_empty(st), par, abort_flag, a.err)) { ok = false; break; }
-        const int jg = jb0 + j;
-        const CUtensorMap* mk;
-        const CUtensorMap* mv;
-        int row;
-        if (jg < nbp) {
-          mk = &mapKp; mv = &mapVp;
-          row = (b * a.Hkv + g) * a.P + (a.P - a.n_vis) + jg * kBN;
-        } else {
-          mk = &mapKc; mv = &mapVc;
-          row = (b * a.Hkv + g) * a.Tc + (jg - nbp) * kBN;
-        }
-        mbar_arrive_expect_tx(kv_full(st), (uint32_t)(2 * L::kKV));
-        for (int c = 0; c < DH / 64; ++c) {
-          tma_load_2d(sbase + L::kKOff + st * L::kKV + c * (kBN * 128), mk, kv_full(st), c * 64, row);
-          tma_load_2d(sbase + L::kVOff + st * L::kKV + c * (kBN * 128), mv, kv_full(st), c * 64, row);
-        }
+        issue_kv(j);
         ++issued;
       }
       if (!ok) {  // abort path: let issued copies land

@@ -166,14 +166,30 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // Everything above overlaps the previous kernel's tail.  The weights do not
-  // depend on it: in DENSE and HEAD the producer issues the weight operand of
-  // its first tile's first stages now (fresh barriers, no empty waits), and
-  // only the activation operand after the wait below.
+  // Everything above overlaps the previous kernel's tail.
+  //
+  // The group tables of the grouped modes come from the router, two or three
+  // kernels back.  The router, the row gather and the gate/up GEMM each call
+  // griddepcontrol.launch_dependents only after their own grid wait, so the
+  // router had completed before the kernel just before this one let it
+  // launch: the tables are read before this kernel's wait.
+  int* s_prefix = reinterpret_cast<int*>(smem + (size_t)S * a.stage_bytes + 1024);
+  int* s_offsets = s_prefix + (a.n_groups + 1);
+  float* s_stage_out = reinterpret_cast<float*>(smem + (size_t)S * a.stage_bytes + 1024 + a.tab_bytes);
+  const bool grouped = a.mode == GEMM_GATEUP || a.mode == GEMM_DOWN;
+  if (grouped) {
+    for (int i = threadIdx.x; i <= a.n_groups; i += blockDim.x) {
+      s_prefix[i] = __ldcg(a.chunk_prefix + i);
+      s_offsets[i] = __ldcg(a.offsets + i);
+    }
+    __syncthreads();
+  }
+  // The weights do not depend on the previous kernel either: the producer
+  // issues the weight operand of its first tile's first stages now (fresh
+  // barriers, no empty waits), and the activation operand after the wait.
   int pre = 0;
-  if (warp == 0 && lane == 0 && (a.mode == GEMM_DENSE || a.mode == GEMM_HEAD) &&
-      (int)blockIdx.x < tile_count(a, nullptr)) {
-    const TileInfo ti = decode_tile(a, blockIdx.x, nullptr, nullptr);
+  if (warp == 0 && lane == 0 && (int)blockIdx.x < tile_count(a, s_prefix)) {
+    const TileInfo ti = decode_tile(a, blockIdx.x, s_prefix, s_offsets);
     const uint32_t tx = (uint32_t)(ti.n_acc * kATileBytes) +
                         (uint32_t)(ti.n_bbox * a.b_box_rows * 128);
     pre = min(S, ti.kb1 - ti.kb0);
@@ -184,30 +200,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       if (a.mode == GEMM_DENSE) {
         for (int i = 0; i < ti.n_acc; ++i)
           tma_load_2d(sA + i * kATileBytes, &mapA, full_bar(p), kx, ti.a_row0 + i * 128);
-      } else {
+      } else if (a.mode == GEMM_HEAD) {
         tma_load_2d(sA + (uint32_t)a.a_bytes, &mapB, full_bar(p), kx, ti.row0);
+      } else {
+        tma_load_3d(sA, &mapA, full_bar(p), kx, ti.a_row0, ti.g);
       }
     }
   }
   // Data written by the previous kernel is read from here on.  A DOWN launch
   // with ready counters does not wait for the whole gate/up grid: its H rows
-  // are guarded per chunk below, and what else it reads (the group tables)
-  // was complete before the gate/up grid let it launch.
+  // are guarded per chunk below.
   const bool handover = a.mode == GEMM_DOWN && a.chunk_ready != nullptr;
   if (!handover) griddep_wait();
   griddep_launch();
-
-  // group tables (written by the router, the kernel before) into shared memory
-  int* s_prefix = reinterpret_cast<int*>(smem + (size_t)S * a.stage_bytes + 1024);
-  int* s_offsets = s_prefix + (a.n_groups + 1);
-  float* s_stage_out = reinterpret_cast<float*>(smem + (size_t)S * a.stage_bytes + 1024 + a.tab_bytes);
-  if (a.mode == GEMM_GATEUP || a.mode == GEMM_DOWN) {
-    for (int i = threadIdx.x; i <= a.n_groups; i += blockDim.x) {
-      s_prefix[i] = __ldcg(a.chunk_prefix + i);
-      s_offsets[i] = __ldcg(a.offsets + i);
-    }
-    __syncthreads();
-  }
 
   const int n_tiles = tile_count(a, s_prefix);
   // TMEM layout: n_bufs tile buffers of 512/n_bufs columns; in a buffer,
@@ -259,7 +264,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
           } else if (a.mode == GEMM_HEAD) {
             for (int i = 0; i < ti.n_acc; ++i)
               tma_load_2d(sA + i * kATileBytes, &mapA, fb, kx, ti.a_row0 + i * 128);
-          } else {
+          } else if (!weight_issued) {
             tma_load_3d(sA, &mapA, fb, kx, ti.a_row0, ti.g);
           }
           if (!(weight_issued && a.mode == GEMM_HEAD))

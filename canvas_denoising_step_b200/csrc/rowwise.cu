@@ -435,38 +435,63 @@ __device__ __forceinline__ void merge_stats(float& m, float& s, int& a, float m2
 }
 }  // namespace
 
-__global__ void head_merge_kernel(const float* hm, const float* hs, const int* ha, int n_vblocks,
-                                  int T, float* conf, int32_t* tok) {
+// A CTA takes 32 token rows (lane = row) and its 32 warps split the vocab
+// blocks into contiguous slices, so that each load instruction reads 32
+// consecutive rows of one block; warp 0 then merges the 32 slices of each row
+// in slice order (the argmax tie rule, lowest index, does not depend on the
+// order; the sum is taken in a fixed order).
+constexpr int kMergeWarps = 32;
+
+__global__ void __launch_bounds__(kMergeWarps * 32) head_merge_kernel(
+    const float* hm, const float* hs, const int* ha, int n_vblocks, int T, float* conf,
+    int32_t* tok) {
+  __shared__ float s_m[kMergeWarps][32], s_s[kMergeWarps][32];
+  __shared__ int s_a[kMergeWarps][32];
   griddep_wait();
   griddep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (t >= T) return;
-  float m = -INFINITY, s = 0.f;
-  int a = 0x7fffffff;
-  const int per = (n_vblocks + 31) / 32;
-  const int v0 = lane * per, v1 = min(n_vblocks, v0 + per);
-  for (int vb = v0; vb < v1; ++vb) {
-    const size_t o = (size_t)vb * T + t;
-    merge_stats(m, s, a, hm[o], hs[o], ha[o]);
-  }
+  const int t = blockIdx.x * 32 + lane;
+  float m = -INFINITY, sum = 0.f;
+  int arg = 0x7fffffff;
+  if (t < T) {
+    const int per = (n_vblocks + kMergeWarps - 1) / kMergeWarps;
+    const int v0 = warp * per, v1 = min(n_vblocks, v0 + per);
+    int vb = v0;
+    for (; vb + 4 <= v1; vb += 4) {   // four blocks' loads in flight
+      float mm[4], ss[4];
+      int aa[4];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
-    const int a2 = __shfl_xor_sync(0xffffffffu, a, o);
-    merge_stats(m, s, a, m2, s2, a2);
+      for (int u = 0; u < 4; ++u) {
+        const size_t o = (size_t)(vb + u) * T + t;
+        mm[u] = hm[o];
+        ss[u] = hs[o];
+        aa[u] = ha[o];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) merge_stats(m, sum, arg, mm[u], ss[u], aa[u]);
+    }
+    for (; vb < v1; ++vb) {
+      const size_t o = (size_t)vb * T + t;
+      merge_stats(m, sum, arg, hm[o], hs[o], ha[o]);
+    }
   }
-  if (lane == 0) {
-    conf[t] = 1.0f / s;
-    tok[t] = a;
+  s_m[warp][lane] = m;
+  s_s[warp][lane] = sum;
+  s_a[warp][lane] = arg;
+  __syncthreads();
+  if (warp == 0 && t < T) {
+    float mt = -INFINITY, st = 0.f;
+    int at = 0x7fffffff;
+    for (int w = 0; w < kMergeWarps; ++w) merge_stats(mt, st, at, s_m[w][lane], s_s[w][lane], s_a[w][lane]);
+    conf[t] = 1.0f / st;
+    tok[t] = at;
   }
 }
 
 cudaError_t launch_head_merge(const float* hm, const float* hs, const int* ha, int n_vblocks,
                               int T, float* conf, int32_t* tok, cudaStream_t s) {
-  return launch_k(head_merge_kernel, dim3((T + 7) / 8), dim3(256), 0, s, hm, hs, ha, n_vblocks, T,
-                  conf, tok);
+  return launch_k(head_merge_kernel, dim3((T + 31) / 32), dim3(kMergeWarps * 32), 0, s, hm, hs,
+                  ha, n_vblocks, T, conf, tok);
 }
 
 // ---------------------------------------------------------------- commit
