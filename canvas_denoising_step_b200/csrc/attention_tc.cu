@@ -54,7 +54,8 @@ template <int DH>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapKc,
                const __grid_constant__ CUtensorMap mapVc, const __grid_constant__ CUtensorMap mapKp,
-               const __grid_constant__ CUtensorMap mapVp, const AttnTcArgs a) {
+               const __grid_constant__ CUtensorMap mapVp, const __grid_constant__ CUtensorMap mapPo,
+               const AttnTcArgs a) {
   using L = AttnSmem<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -299,8 +300,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
       R = ((size_t)b * a.Hq + h) * a.Tc + i;
     }
     float* po = a.part_o + ((size_t)chunk * rows_total + R) * DH;
+    // The partial O leaves through shared memory: this warp stages its 32 rows
+    // x 32 columns (128-byte swizzle: float4 c of row r at c ^ (r % 8)) in the
+    // K/V ring, idle now, and lane 0 writes the block with a tensor store.
+    // The 32 rows are consecutive in part_o when all are valid (R = R0 + qr);
+    // otherwise the valid ones are written directly.
+    const bool warp_full = __all_sync(0xffffffffu, row_valid);
+    const int row0 = chunk * rows_total + (b * a.Hq + g * group) * a.Tc + qt * kRows + q * 32;
+    const uint32_t stage_base = sbase + L::kKOff + (uint32_t)(warp - 2) * 8192u;
 #pragma unroll 1
-    for (int c0 = 0; c0 < DH; c0 += 32) {
+    for (int c0 = 0, sbuf = 0; c0 < DH; c0 += 32, sbuf ^= 1) {
       if (n_local > 0 && ok) {
         tmem_ld32(lane_base + kOCol + c0, v);
         tmem_wait_ld();
@@ -308,7 +317,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = 0u;
       }
-      if (row_valid) {
+      if (warp_full) {
+        const uint32_t st = stage_base + (uint32_t)sbuf * 4096u;
+        if (lane == 0) bulk_wait_read<1>();   // the store that last read this buffer is done
+        __syncwarp();
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4)
+          st_shared_v4(st + (uint32_t)lane * 128u + (uint32_t)((c4 ^ (lane & 7)) * 16),
+                       v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&mapPo, st, c0, row0);
+          bulk_commit();
+        }
+      } else if (row_valid) {
 #pragma unroll
         for (int e = 0; e < 32; e += 4)
           *reinterpret_cast<float4*>(po + c0 + e) =
@@ -316,6 +339,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                           __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
       }
     }
+    if (warp_full && lane == 0) bulk_wait_all();
+    __syncwarp();
     if (row_valid) {
       float* pml = a.part_ml + ((size_t)chunk * rows_total + R) * 2;
       pml[0] = (n_local > 0) ? m : -INFINITY;
@@ -345,7 +370,8 @@ cudaError_t launch_attn_tc_t(const AttnTcMaps& m, const AttnTcArgs& a, cudaStrea
   }
   const int group = a.Hq / a.Hkv;
   dim3 grid((group * a.Tc + kRows - 1) / kRows, a.n_chunks, a.B * a.Hkv);
-  return launch_k(attn_tc_kernel<DH>, grid, dim3(kThreads), smem, s, m.q, m.kc, m.vc, m.kp, m.vp, a);
+  return launch_k(attn_tc_kernel<DH>, grid, dim3(kThreads), smem, s, m.q, m.kc, m.vc, m.kp, m.vp,
+                  m.po, a);
 }
 
 }  // namespace

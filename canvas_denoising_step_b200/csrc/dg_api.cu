@@ -86,6 +86,7 @@ struct dg_ctx {
   CUtensorMap m_x_b, m_x_a, m_attn_o_b, m_xperm_b, m_H_b, m_x2_b;
   CUtensorMap m_Y_out;   // fp32 expert outputs [1][rows][d], tensor-store map
   CUtensorMap m_q, m_kc, m_vc;   // attention operands
+  CUtensorMap m_attn_po;         // attention partial outputs (tensor stores)
 
   int last_T = 0, last_B = 0, launches = 0;
   int* steps_dev = nullptr;          // steps_left of the pass being run
@@ -303,6 +304,7 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
   ta.err = c->err_dev;
   AttnTcMaps tm;
   tm.q = c->m_q; tm.kc = c->m_kc; tm.vc = c->m_vc; tm.kp = L.m_kp; tm.vp = L.m_vp;
+  tm.po = c->m_attn_po;
   DG_LAUNCH(c, K_ATTN, launch_attention_tc(tm, ta, c->stream));
   AttnArgs at;   // the merge reads the partials' shape from here
   memset(&at, 0, sizeof(at));
@@ -602,6 +604,7 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
   ok &= make_tmap_2d(&c->m_H_b, c->H, F, rows_moe, kGroupedBox);
   ok &= make_tmap_out_f32(&c->m_Y_out, c->Y, d, rows_moe, 1);
   ok &= make_tmap_2d(&c->m_q, c->q, dh, std::max<size_t>(T * Hq, 128), 128);
+  ok &= make_tmap_f32_sw128(&c->m_attn_po, c->attn_po, dh, (uint64_t)kMaxAttnChunks * T * Hq);
   ok &= make_tmap_2d(&c->m_kc, c->kc, dh, std::max<size_t>(T * Hkv, 64), 64);
   ok &= make_tmap_2d(&c->m_vc, c->vc, dh, std::max<size_t>(T * Hkv, 64), 64);
   if (cudaDeviceSynchronize() != cudaSuccess || !ok) {

@@ -43,6 +43,9 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t o
                   uint32_t box_outer);
 bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid,
                   uint64_t outer, uint32_t box_mid);
+// fp32 [outer][inner] map with 32 x 32 boxes in the 128-byte swizzle (the
+// attention's partial-output stores).
+bool make_tmap_f32_sw128(CUtensorMap* map, float* base, uint64_t inner, uint64_t outer);
 // fp32 [outer][mid][inner] output map for the DENSE / DOWN tensor stores.
 bool make_tmap_out_f32(CUtensorMap* map, float* base, uint64_t inner, uint64_t mid,
                        uint64_t outer);
@@ -128,6 +131,7 @@ struct AttnTcMaps {
   CUtensorMap q;         // [B*Hq*Tc][dh], box 64 x 128 rows
   CUtensorMap kc, vc;    // [B*Hkv*Tc][dh], box 64 x 64 rows
   CUtensorMap kp, vp;    // [B*Hkv*P][dh],  box 64 x 64 rows
+  CUtensorMap po;        // part_o as [chunks * rows][dh] fp32, box 32 x 32, 128-byte swizzle
 };
 int attn_tc_blocks(int n_vis, int Tc);
 int attn_tc_qtiles(int Hq, int Hkv, int Tc);

@@ -515,6 +515,20 @@ bool make_tmap_out_f32(CUtensorMap* map, float* base, uint64_t inner, uint64_t m
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 [outer][inner] written in 32 x 32 blocks whose shared-memory image has
+// the 128-byte swizzle (16-byte chunk c of row r at chunk c ^ (r % 8)).
+bool make_tmap_f32_sw128(CUtensorMap* map, float* base, uint64_t inner, uint64_t outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Shared-memory plan: A region (1 or 2 tiles of 16 KB) + B region, as many
 // stages as fit beside the barriers, group tables and output staging; and the
 // TMEM plan: two tile buffers of 256
