@@ -85,6 +85,7 @@ struct dg_ctx {
   bool has_bias = false;
   CUtensorMap m_x_b, m_x_a, m_attn_o_b, m_xperm_b, m_H_b, m_x2_b;
   CUtensorMap m_Y_out;   // fp32 expert outputs [1][rows][d], tensor-store map
+  CUtensorMap m_H_out;   // bf16 gate/up outputs [rows][F], tensor-store map
   CUtensorMap m_q, m_kc, m_vc;   // attention operands
   CUtensorMap m_attn_po;         // attention partial outputs (tensor stores)
 
@@ -269,7 +270,8 @@ int run_grouped(dg_ctx* c, int mode, const CUtensorMap& mA, const CUtensorMap& m
   (void)T;
   gemm_plan_smem(a);
   DG_LAUNCH(c, mode == GEMM_GATEUP ? K_GEMM_GATEUP : K_GEMM_DOWN,
-            gemm_tc_launch(mA, mB, c->m_Y_out, a, c->num_sms, c->stream));
+            gemm_tc_launch(mA, mB, mode == GEMM_GATEUP ? c->m_H_out : c->m_Y_out, a, c->num_sms,
+                           c->stream));
   return DG_OK;
 }
 
@@ -603,6 +605,7 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
   ok &= make_tmap_2d(&c->m_x2_b, c->xperm, d, rows_moe, c->dense_box);
   ok &= make_tmap_2d(&c->m_H_b, c->H, F, rows_moe, kGroupedBox);
   ok &= make_tmap_out_f32(&c->m_Y_out, c->Y, d, rows_moe, 1);
+  ok &= make_tmap_h_store(&c->m_H_out, c->H, F, rows_moe);
   ok &= make_tmap_2d(&c->m_q, c->q, dh, std::max<size_t>(T * Hq, 128), 128);
   ok &= make_tmap_f32_sw128(&c->m_attn_po, c->attn_po, dh, (uint64_t)kMaxAttnChunks * T * Hq);
   ok &= make_tmap_2d(&c->m_kc, c->kc, dh, std::max<size_t>(T * Hkv, 64), 64);

@@ -43,6 +43,8 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t o
                   uint32_t box_outer);
 bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid,
                   uint64_t outer, uint32_t box_mid);
+// bf16 [outer][inner] map with [32 rows][16] boxes (the gate/up H stores).
+bool make_tmap_h_store(CUtensorMap* map, void* base, uint64_t inner, uint64_t outer);
 // fp32 [outer][inner] map with 32 x 32 boxes in the 128-byte swizzle (the
 // attention's partial-output stores).
 bool make_tmap_f32_sw128(CUtensorMap* map, float* base, uint64_t inner, uint64_t outer);
@@ -51,8 +53,8 @@ bool make_tmap_out_f32(CUtensorMap* map, float* base, uint64_t inner, uint64_t m
                        uint64_t outer);
 void gemm_plan_smem(GemmArgs& a);
 size_t gemm_smem_bytes(const GemmArgs& a);
-// mapC: the fp32 output map (DENSE: [k_splits][N][M]; DOWN: [1][rows][M]); any
-// valid map for the other modes, which do not use it.
+// mapC: the output map (DENSE: fp32 [k_splits][N][M]; DOWN: fp32 [1][rows][M];
+// GATEUP: bf16 H [rows][F]); any valid map for HEAD, which does not use it.
 cudaError_t gemm_tc_launch(const CUtensorMap& mapA, const CUtensorMap& mapB,
                            const CUtensorMap& mapC, const GemmArgs& a, int grid,
                            cudaStream_t stream);

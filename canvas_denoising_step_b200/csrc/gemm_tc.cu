@@ -380,22 +380,56 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       } else if (a.mode == GEMM_GATEUP) {
         // Interleaved rows: even accumulator rows are gate rows, odd rows the
         // matching up rows of the same output feature f.
+        // A warp's 16 gate rows are 16 consecutive features f0 .. f0+15; a full
+        // 32-row chunk of H leaves as one [32 rows][16 f] bf16 block through
+        // shared memory and a tensor store (lanes 4p pack f0+2p, f0+2p+1);
+        // a chunk that ends inside the group's rows is stored element-wise.
         const int f = (ti.m_slab * 128 + r) >> 1;
+        const int f0 = (ti.m_slab * 128 + q * 32) >> 1;
         const bool is_gate = (r & 1) == 0;
+        const uint32_t h_stage = smem_u32(s_stage_out) + (uint32_t)(warp - 2) * 2048u;
         for (int c0 = 0; c0 < ti.n_mma; c0 += 32) {
           tmem_ld32(lane_addr + (uint32_t)c0, v);
           tmem_wait_ld();
+          if (c0 + 32 <= ti.rows && f0 + 16 <= a.F) {
+            const uint32_t st = h_stage + (uint32_t)sbuf * 1024u;
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float x = __uint_as_float(v[j]);
-            const float u = __shfl_xor_sync(0xffffffffu, x, 1);
-            const int n = c0 + j;
-            if (is_gate && n < ti.rows && f < a.F) {
-              const float h = x / (1.0f + __expf(-x)) * u;
-              a.out_bf16[(size_t)(ti.row0 + n) * a.F + f] = f_to_bf16(h);
+            for (int j = 0; j < 32; ++j) {
+              const float x = __uint_as_float(v[j]);
+              const float u = __shfl_xor_sync(0xffffffffu, x, 1);
+              const float h = x / (1.0f + __expf(-x)) * u;       // meaningful in gate lanes
+              const float h1 = __shfl_down_sync(0xffffffffu, h, 2);  // feature f + 1
+              if ((lane & 3) == 0) {
+                __nv_bfloat162 p2 = __floats2bfloat162_rn(h, h1);
+                st_shared_b32(st + (uint32_t)j * 32u + (uint32_t)(lane >> 2) * 4u,
+                              *reinterpret_cast<uint32_t*>(&p2));
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&mapC, st, f0, ti.row0 + c0);
+              bulk_commit();
+            }
+            sbuf ^= 1;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float x = __uint_as_float(v[j]);
+              const float u = __shfl_xor_sync(0xffffffffu, x, 1);
+              const int n = c0 + j;
+              if (is_gate && n < ti.rows && f < a.F) {
+                const float h = x / (1.0f + __expf(-x)) * u;
+                a.out_bf16[(size_t)(ti.row0 + n) * a.F + f] = f_to_bf16(h);
+              }
             }
           }
         }
+        // the tensor stores of this tile's H have completed before the count
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
         if (a.chunk_ready) {
           // this warp's H writes of the tile are visible before the count
           __threadfence();
@@ -515,6 +549,19 @@ bool make_tmap_out_f32(CUtensorMap* map, float* base, uint64_t inner, uint64_t m
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 [outer][inner] written in [32 rows][16] blocks (the gate/up H stores).
+bool make_tmap_h_store(CUtensorMap* map, void* base, uint64_t inner, uint64_t outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {16, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // fp32 [outer][inner] written in 32 x 32 blocks whose shared-memory image has
 // the 128-byte swizzle (16-byte chunk c of row r at chunk c ^ (r % 8)).
 bool make_tmap_f32_sw128(CUtensorMap* map, float* base, uint64_t inner, uint64_t outer) {
@@ -541,7 +588,8 @@ void gemm_plan_smem(GemmArgs& a) {
   // DENSE, one for DOWN (which keeps its sixth operand stage)
   a.tab_bytes = (a.mode == GEMM_GATEUP || a.mode == GEMM_DOWN)
                     ? ((2 * (a.n_groups + 1) * 4 + 127) / 128) * 128 : 0;
-  a.epi_bytes = a.mode == GEMM_DENSE ? 2 * 4 * 4096 : (a.mode == GEMM_DOWN ? 4 * 4096 : 0);
+  a.epi_bytes = a.mode == GEMM_DENSE ? 2 * 4 * 4096
+                : (a.mode == GEMM_DOWN ? 4 * 4096 : (a.mode == GEMM_GATEUP ? 2 * 4 * 1024 : 0));
   a.a_bytes = n_a * kATileBytes;
   if (a.mode == GEMM_HEAD) {
     a.b_box_rows = 256;
