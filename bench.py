@@ -300,6 +300,22 @@ def run_reference(args, cfg, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(values, world, device):
+    """Each timing taken as the maximum over the ranks (the slowest replica)."""
+    if world == 1:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def canvas_throughput(world, batch, canvas_len, steps, steps_per_block, t_ms):
+    """Whole-job canvas tokens/s: every replica finalises batch * canvas_len tokens per
+    steps_per_block passes; `steps` passes took t_ms (max over ranks)."""
+    return world * batch * canvas_len * steps / steps_per_block / (t_ms / 1e3)
+
+
 def run_ours(args, cfg, rank, world, local_rank):
     import torch
     import canvas_denoising_step_b200 as dg
@@ -389,17 +405,12 @@ def run_ours(args, cfg, rank, world, local_rank):
         ms_e2e = f0.elapsed_time(f1)
         barrier()
 
-    t_max, t_e2e_max = ms, ms_e2e
-    if world > 1:
-        t = torch.tensor([ms, ms_e2e], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        t_max, t_e2e_max = float(t[0]), float(t[1])
+    t_max, t_e2e_max = max_over_ranks([ms, ms_e2e], world, dev)
     dg.dg_destroy(ctx)
     if rank != 0:
         return
 
-    tokens = world * B * Tc * args.steps / S
-    value = tokens / (t_max / 1e3)
+    value = canvas_throughput(world, B, Tc, args.steps, S, t_max)
     peak, peak_kind = load_peaks()
     gu_ms, gu_n = kern.get("gemm_gateup", (float("nan"), 1))
     gu_bytes = gateup_bytes_per_launch(cfg, active_avg)
@@ -428,7 +439,8 @@ def run_ours(args, cfg, rank, world, local_rank):
                                 sorted(kern.items(), key=lambda kv: -kv[1][0])},
         "profiled_ms_per_step": total_prof / args.steps,
         "gpu_launches": launches_per_step * args.steps,
-        "e2e": {"value": tokens / (t_e2e_max / 1e3), "unit": "canvas tokens/s",
+        "e2e": {"value": canvas_throughput(world, B, Tc, args.steps, S, t_e2e_max),
+                "unit": "canvas tokens/s",
                 "h2d_bytes_per_step": T * 4, "d2h_bytes_per_step": T * 4 + T * 4 + T},
         "clocks": clk,
     }
