@@ -10,7 +10,7 @@ namespace dg {
 namespace {
 
 template <int DH>
-__global__ void attn_merge_kernel(const AttnArgs a, bf16* out) {
+__global__ void attn_merge_kernel(const AttnMergeArgs a, bf16* out) {
   griddep_wait();
   griddep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -47,7 +47,7 @@ __global__ void attn_merge_kernel(const AttnArgs a, bf16* out) {
 
 }  // namespace
 
-cudaError_t launch_attn_merge(const AttnArgs& a, bf16* o, cudaStream_t s) {
+cudaError_t launch_attn_merge(const AttnMergeArgs& a, bf16* o, cudaStream_t s) {
   const int rows = a.B * a.Hq * a.Tc;
   const int grid = (rows + 7) / 8;
   switch (a.dh) {

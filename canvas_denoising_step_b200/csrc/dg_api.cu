@@ -308,9 +308,8 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
   tm.q = c->m_q; tm.kc = c->m_kc; tm.vc = c->m_vc; tm.kp = L.m_kp; tm.vp = L.m_vp;
   tm.po = c->m_attn_po;
   DG_LAUNCH(c, K_ATTN, launch_attention_tc(tm, ta, c->stream));
-  AttnArgs at;   // the merge reads the partials' shape from here
-  memset(&at, 0, sizeof(at));
-  at.B = B; at.Hq = Hq; at.Hkv = Hkv; at.Tc = Tc; at.P = P; at.dh = dh;
+  AttnMergeArgs at;
+  at.B = B; at.Hq = Hq; at.Tc = Tc; at.dh = dh;
   at.n_chunks = ta.n_chunks;
   at.part_o = c->attn_po; at.part_ml = c->attn_ml;
   DG_LAUNCH(c, K_ATTN_MERGE, launch_attn_merge(at, c->attn_o, c->stream));

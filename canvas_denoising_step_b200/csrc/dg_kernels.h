@@ -102,23 +102,18 @@ cudaError_t launch_qkv_rope(const float* part, int splits, int T, int Tc, int Hq
                             int n_rot, const float* cos_t, const float* sin_t, bf16* q, bf16* kc,
                             bf16* vc, cudaStream_t s);
 
-// Shape of the split-KV attention partials (read by the merge).
-struct AttnArgs {
-  const bf16* q;   // [B][Hq][Tc][dh]
-  const bf16* kc;  // [B][Hkv][Tc][dh]
-  const bf16* vc;
-  const bf16* kp;  // [B][Hkv][P][dh]
-  const bf16* vp;
-  int B, Hq, Hkv, Tc, P, dh;
-  int n_vis;       // visible prompt keys (the last n_vis)
-  int n_chunks, chunk_keys;
-  float* part_o;   // [n_chunks][B*Hq*Tc][dh]
-  float* part_ml;  // [n_chunks][B*Hq*Tc][2]  (max in log2 units, sum)
-  float scale_log2;  // log2(e) / sqrt(dh)
+// The split-KV attention partials, as the merge reads them: per key-range
+// chunk c and query row R = (b * Hq + h) * Tc + i, the un-normalised O
+// (part_o[c][R][dh]) and (m, l) with m in log2 units (part_ml[c][R][2]).
+struct AttnMergeArgs {
+  int B, Hq, Tc, dh;
+  int n_chunks;
+  const float* part_o;   // [n_chunks][B*Hq*Tc][dh]
+  const float* part_ml;  // [n_chunks][B*Hq*Tc][2]
 };
 
 // tcgen05 attention (attention_tc.cu): writes the split-KV partials part_o /
-// part_ml in the AttnArgs layout above; launch_attn_merge (attn_merge.cu)
+// part_ml in the AttnMergeArgs layout above; launch_attn_merge (attn_merge.cu)
 // combines them.
 struct AttnTcArgs {
   int B, Hq, Hkv, Tc, P, dh;
@@ -139,7 +134,7 @@ int attn_tc_blocks(int n_vis, int Tc);
 int attn_tc_qtiles(int Hq, int Hkv, int Tc);
 cudaError_t launch_attention_tc(const AttnTcMaps& m, const AttnTcArgs& a, cudaStream_t s);
 // Merge partials -> o [T][Hq*dh] bf16 (t = b*Tc + i)
-cudaError_t launch_attn_merge(const AttnArgs& a, bf16* o, cudaStream_t s);
+cudaError_t launch_attn_merge(const AttnMergeArgs& a, bf16* o, cudaStream_t s);
 
 // a = sum of O-projection partials; h1 = h + rmsnorm(a)*w_post (h updated in
 // place); x2 = bf16(rmsnorm(h1)*w_ff).

@@ -4,7 +4,7 @@ Tolerances: bf16 layer outputs within relative L2 1e-2; router indices,
 permutations and commit decisions bit-exact when both sides see identical
 scores (ties toward the lower index).  Intermediate stages are checked with
 teacher forcing: the oracle step is fed the device's own input to that step,
-so each kernel is judged alone.
+so each kernel is checked alone.
 """
 
 import numpy as np
