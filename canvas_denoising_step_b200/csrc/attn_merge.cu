@@ -11,30 +11,52 @@ namespace {
 
 template <int DH>
 __global__ void attn_merge_kernel(const AttnMergeArgs a, bf16* out) {
+  constexpr int NJ = DH / 64;   // float2 per lane per chunk: lane covers 2 * lane + 64 * j
+  constexpr int kBatch = 4;     // chunks whose loads are in flight together
   griddep_wait();
   griddep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rows_total = a.B * a.Hq * a.Tc;
   const int R = blockIdx.x * (blockDim.x >> 5) + warp;
   if (R >= rows_total) return;
+  const int nc = a.n_chunks;
   // lane c holds chunk c's (m, l); n_chunks <= 32
   float mc = -INFINITY, lc = 0.f;
-  if (lane < a.n_chunks) {
-    const float2 ml = *reinterpret_cast<const float2*>(a.part_ml + ((size_t)lane * rows_total + R) * 2);
+  if (lane < nc) {
+    const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml + ((size_t)lane * rows_total + R) * 2));
     mc = ml.x;
     lc = ml.y;
   }
-  const float M = warp_max(mc);
-  const float wl = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
-  const float L = warp_sum(wl * lc);
-  float acc[DH / 32];
+  float2 acc[NJ];
 #pragma unroll
-  for (int j = 0; j < DH / 32; ++j) acc[j] = 0.f;
-  for (int c = 0; c < a.n_chunks; ++c) {
-    const float wgt = __shfl_sync(0xffffffffu, wl, c);
-    const float* po = a.part_o + ((size_t)c * rows_total + R) * DH;
+  for (int j = 0; j < NJ; ++j) acc[j] = make_float2(0.f, 0.f);
+  float M = 0.f, wl = 0.f, L = 0.f;
+  for (int c0 = 0; c0 < nc; c0 += kBatch) {
+    // the partial O of up to kBatch chunks, loaded before they are needed
+    float2 buf[kBatch][NJ];
 #pragma unroll
-    for (int j = 0; j < DH / 32; ++j) acc[j] += wgt * po[lane + 32 * j];
+    for (int u = 0; u < kBatch; ++u)
+#pragma unroll
+      for (int j = 0; j < NJ; ++j)
+        buf[u][j] = (c0 + u < nc)
+                        ? __ldcg(reinterpret_cast<const float2*>(
+                              a.part_o + ((size_t)(c0 + u) * rows_total + R) * DH + 2 * lane + 64 * j))
+                        : make_float2(0.f, 0.f);
+    if (c0 == 0) {
+      M = warp_max(mc);
+      wl = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+      L = warp_sum(wl * lc);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const float wgt = __shfl_sync(0xffffffffu, wl, (c0 + u) & 31);
+      if (c0 + u < nc)
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+          acc[j].x += wgt * buf[u][j].x;
+          acc[j].y += wgt * buf[u][j].y;
+        }
+    }
   }
   const int i = R % a.Tc;
   const int bh = R / a.Tc;
@@ -42,7 +64,9 @@ __global__ void attn_merge_kernel(const AttnMergeArgs a, bf16* out) {
   bf16* dst = out + ((size_t)b * a.Tc + i) * ((size_t)a.Hq * DH) + (size_t)h * DH;
   const float inv = 1.0f / L;
 #pragma unroll
-  for (int j = 0; j < DH / 32; ++j) dst[lane + 32 * j] = f_to_bf16(acc[j] * inv);
+  for (int j = 0; j < NJ; ++j)
+    *reinterpret_cast<__nv_bfloat162*>(dst + 2 * lane + 64 * j) =
+        __floats2bfloat162_rn(acc[j].x * inv, acc[j].y * inv);
 }
 
 }  // namespace

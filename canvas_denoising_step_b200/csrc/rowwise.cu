@@ -159,11 +159,15 @@ cudaError_t launch_rope_table(float* cos_t, float* sin_t, int Tc, int half, int 
 
 // ---------------------------------------------------------------- q/k/v split-K sum + RoPE
 
-// One CTA per canvas row.  Work item p = (head hh, 4-pair group j4): pairs
-// (j, j + dh/2) for j = 4*j4 .. 4*j4+3, loaded as two float4 per split.
-constexpr int kRopeItems = 8;  // items per thread: (Hq + 2 Hkv) * dh / 8 <= 2048
+// A CTA takes one canvas row and up to kRopeThreads * kRopeItems work items of
+// it (a second grid dimension covers wider rows).  Work item p = (head hh,
+// 4-pair group j4): pairs (j, j + dh/2) for j = 4*j4 .. 4*j4+3, loaded as two
+// float4 per split, two splits' loads in flight at once.  Four items per
+// thread keep the registers low enough for two CTAs per SM.
+constexpr int kRopeItems = 4;
+constexpr int kRopeThreads = 256;
 
-__global__ void __launch_bounds__(kRowThreads) qkv_rope_kernel(
+__global__ void __launch_bounds__(kRopeThreads, 2) qkv_rope_kernel(
     const float* part, int splits, int T, int Tc, int Hq, int Hkv, int dh, int n_rot,
     const float* cos_t, const float* sin_t, bf16* q, bf16* kc, bf16* vc) {
   griddep_wait();
@@ -173,30 +177,38 @@ __global__ void __launch_bounds__(kRowThreads) qkv_rope_kernel(
   const int nqkv = (Hq + 2 * Hkv) * dh;
   const int half = dh / 2, q4 = half / 4;
   const int n_items = (Hq + 2 * Hkv) * q4;
+  const int p0 = blockIdx.y * kRopeThreads * kRopeItems + threadIdx.x;
   float4 x0[kRopeItems], x1[kRopeItems];
 #pragma unroll
   for (int u = 0; u < kRopeItems; ++u) x0[u] = x1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < splits; ++s) {
-    const float* src = part + ((size_t)s * T + t) * nqkv;
-    float4 a[kRopeItems], c[kRopeItems];
+  for (int s0 = 0; s0 < splits; s0 += 2) {
+    float4 a[2][kRopeItems], c[2][kRopeItems];
 #pragma unroll
-    for (int u = 0; u < kRopeItems; ++u) {
-      const int p = threadIdx.x + kRowThreads * u;
-      if (p < n_items) {
-        const int hh = p / q4, j = (p % q4) * 4;
-        a[u] = __ldg(reinterpret_cast<const float4*>(src + hh * dh + j));
-        c[u] = __ldg(reinterpret_cast<const float4*>(src + hh * dh + j + half));
+    for (int ss = 0; ss < 2; ++ss) {
+      const float* src = part + ((size_t)(s0 + ss) * T + t) * nqkv;
+#pragma unroll
+      for (int u = 0; u < kRopeItems; ++u) {
+        const int p = p0 + kRopeThreads * u;
+        if (s0 + ss < splits && p < n_items) {
+          const int hh = p / q4, j = (p % q4) * 4;
+          a[ss][u] = __ldcg(reinterpret_cast<const float4*>(src + hh * dh + j));
+          c[ss][u] = __ldcg(reinterpret_cast<const float4*>(src + hh * dh + j + half));
+        } else {
+          a[ss][u] = c[ss][u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
     }
 #pragma unroll
-    for (int u = 0; u < kRopeItems; ++u) {
-      x0[u].x += a[u].x; x0[u].y += a[u].y; x0[u].z += a[u].z; x0[u].w += a[u].w;
-      x1[u].x += c[u].x; x1[u].y += c[u].y; x1[u].z += c[u].z; x1[u].w += c[u].w;
-    }
+    for (int ss = 0; ss < 2; ++ss)
+#pragma unroll
+      for (int u = 0; u < kRopeItems; ++u) {
+        x0[u].x += a[ss][u].x; x0[u].y += a[ss][u].y; x0[u].z += a[ss][u].z; x0[u].w += a[ss][u].w;
+        x1[u].x += c[ss][u].x; x1[u].y += c[ss][u].y; x1[u].z += c[ss][u].z; x1[u].w += c[ss][u].w;
+      }
   }
 #pragma unroll
   for (int u = 0; u < kRopeItems; ++u) {
-    const int p = threadIdx.x + kRowThreads * u;
+    const int p = p0 + kRopeThreads * u;
     if (p >= n_items) continue;
     const int hh = p / q4, j = (p % q4) * 4;
     bf16* dst;
@@ -230,8 +242,10 @@ __global__ void __launch_bounds__(kRowThreads) qkv_rope_kernel(
 cudaError_t launch_qkv_rope(const float* part, int splits, int T, int Tc, int Hq, int Hkv, int dh,
                             int n_rot, const float* cos_t, const float* sin_t, bf16* q, bf16* kc,
                             bf16* vc, cudaStream_t s) {
-  return launch_k(qkv_rope_kernel, dim3(T), dim3(kRowThreads), 0, s, part, splits, T, Tc, Hq, Hkv,
-                  dh, n_rot, cos_t, sin_t, q, kc, vc);
+  const int n_items = (Hq + 2 * Hkv) * (dh / 8);
+  const int per_cta = kRopeThreads * kRopeItems;
+  return launch_k(qkv_rope_kernel, dim3(T, (n_items + per_cta - 1) / per_cta), dim3(kRopeThreads),
+                  0, s, part, splits, T, Tc, Hq, Hkv, dh, n_rot, cos_t, sin_t, q, kc, vc);
 }
 
 // ---------------------------------------------------------------- post-attention norms
