@@ -257,6 +257,13 @@ __global__ void __launch_bounds__(kRowThreads) post_attn_kernel(
   griddep_wait();
   griddep_launch();
   const int t = blockIdx.x, n8 = d / 8;
+  // the residual row goes out first, beside the partials' loads
+  float hv[kChunks][8];
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i) {
+    const int c = threadIdx.x + kRowThreads * i;
+    if (c < n8) ld8f_rw(h + (size_t)t * d + 8 * c, hv[i]);
+  }
   float a[kChunks][8];
 #pragma unroll
   for (int i = 0; i < kChunks; ++i)
@@ -293,12 +300,11 @@ __global__ void __launch_bounds__(kRowThreads) post_attn_kernel(
   for (int i = 0; i < kChunks; ++i) {
     const int c = threadIdx.x + kRowThreads * i;
     if (c >= n8) continue;
-    float hv[8], wv[8];
-    ld8f_rw(h + (size_t)t * d + 8 * c, hv);
+    float wv[8];
     ld8f(w_post + 8 * c, wv);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      a[i][e] = hv[e] + a[i][e] * r1 * wv[e];
+      a[i][e] = hv[i][e] + a[i][e] * r1 * wv[e];
       ss2 += a[i][e] * a[i][e];
     }
     st8f(h + (size_t)t * d + 8 * c, a[i]);
@@ -351,6 +357,13 @@ __global__ void __launch_bounds__(kRowThreads) moe_combine_kernel(
   griddep_wait();
   griddep_launch();
   const int t = blockIdx.x, n8 = d / 8;
+  // the residual row goes out with the routing loads
+  float hv[kChunks][8];
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i) {
+    const int c = threadIdx.x + kRowThreads * i;
+    if (c < n8) ld8f_rw(h + (size_t)t * d + 8 * c, hv[i]);
+  }
   if (threadIdx.x < k) {
     srow[threadIdx.x] = T + inv[(size_t)t * k + threadIdx.x];
     sw[threadIdx.x] = w[(size_t)t * k + threadIdx.x];
@@ -393,11 +406,9 @@ __global__ void __launch_bounds__(kRowThreads) moe_combine_kernel(
   for (int i = 0; i < kChunks; ++i) {
     const int c = threadIdx.x + kRowThreads * i;
     if (c >= n8) continue;
-    float hv[8];
-    ld8f_rw(h + (size_t)t * d + 8 * c, hv);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      y[i][e] += hv[e];
+      y[i][e] += hv[i][e];
       ss += y[i][e] * y[i][e];
     }
     st8f(h + (size_t)t * d + 8 * c, y[i]);
@@ -513,29 +524,38 @@ cudaError_t launch_head_merge(const float* hm, const float* hs, const int* ha, i
 __global__ void commit_kernel(const float* conf, const int32_t* tok, int32_t* canvas,
                               uint8_t* committed, int Tc, int steps_left, const int* steps_dev,
                               int mask_id) {
-  __shared__ float sc[256];
-  __shared__ int sm[256];
+  __shared__ __align__(16) float sc[256];
+  __shared__ __align__(16) int sm[256];
   griddep_wait();
   griddep_launch();
   const int b = blockIdx.x, i = threadIdx.x;
   const size_t o = (size_t)b * Tc;
+  const int sl = steps_left >= 1 ? steps_left : max(1, *steps_dev);
   int masked = 0;
+  float c = -INFINITY;
   if (i < Tc) {
     masked = canvas[o + i] == mask_id;
-    float c = conf[o + i];
+    c = conf[o + i];
     if (c != c) c = -INFINITY;
-    sc[i] = c;
-    sm[i] = masked;
   }
+  sc[i] = c;          // slots past Tc: not masked, never counted
+  sm[i] = masked;
   const int r = __syncthreads_count(masked);
-  const int sl = steps_left >= 1 ? steps_left : max(1, *steps_dev);
   const int k = (r + sl - 1) / sl;
   if (i < Tc) {
     int com = 0;
     if (masked) {
-      const float ci = sc[i];
+      const float ci = c;
       int rank = 0;
-      for (int j = 0; j < Tc; ++j) rank += sm[j] && (sc[j] > ci || (sc[j] == ci && j < i));
+      // four slots per shared-memory load
+      for (int j = 0; j < Tc; j += 4) {
+        const float4 c4 = *reinterpret_cast<const float4*>(sc + j);
+        const int4 m4 = *reinterpret_cast<const int4*>(sm + j);
+        rank += m4.x && (c4.x > ci || (c4.x == ci && j < i));
+        rank += m4.y && (c4.y > ci || (c4.y == ci && j + 1 < i));
+        rank += m4.z && (c4.z > ci || (c4.z == ci && j + 2 < i));
+        rank += m4.w && (c4.w > ci || (c4.w == ci && j + 3 < i));
+      }
       if (rank < k) {
         canvas[o + i] = tok[o + i];
         com = 1;
