@@ -67,6 +67,7 @@ _SIGS = {
     "dg_router_topk": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "dg_router_topk_static": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
                                       c_void_p, c_void_p, c_void_p]),
+    "dg_selftest_bounded_wait": (c_int, [c_void_p]),
     "dg_commit": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p]),
     "dg_debug_tensor": (c_int, [c_void_p, c_char_p, c_void_p, c_size_t, POINTER(c_size_t)]),
     "dg_profile_enable": (c_int, [c_void_p, c_int]),
@@ -156,6 +157,11 @@ def dg_router_topk_static(logits: int, n_rows: int, n_experts: int, top_k: int, 
                                       stream)
     if code != DG_OK:
         raise DgError(code, "dg_router_topk_static", "rejected or failed")
+
+
+def dg_selftest_bounded_wait(stream: int = 0) -> int:
+    """Runs the bounded-wait self-test; returns its status (DG_ERR_TIMEOUT expected)."""
+    return _lib.dg_selftest_bounded_wait(stream)
 
 
 def dg_commit(ctx: int, conf: int, canvas: int, batch: int, steps_left: int, cand_tok: int,

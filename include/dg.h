@@ -182,6 +182,16 @@ int dg_router_topk_static(const float* logits, int n_rows, int n_experts, int to
                           int32_t* idx, float* w, int32_t* offsets, int32_t* perm,
                           void* cuda_stream);
 
+/* Self-test of the bounded waits that every kernel of the library uses (the
+ * device half of the failure detection): runs one CTA on cuda_stream (NULL =
+ * legacy default stream) that waits on an mbarrier nothing arrives on.  The
+ * wait gives up after its limit (2 s), records DG_ERR_TIMEOUT and the kernel
+ * returns, so the device and any context stay usable.  Returns DG_ERR_TIMEOUT
+ * when the wait ran out as designed, DG_OK if it did not run out, DG_ERR_OOM /
+ * DG_ERR_CUDA if the test itself could not run.  Synchronises the stream;
+ * allocates (and frees) one int of device memory. */
+int dg_selftest_bounded_wait(void* cuda_stream);
+
 /* Commit test hook: the commit rule of dg_canvas_step on given confidences.
  * conf: dev fp32 [batch][canvas_len]; cand_tok: dev int32 [batch][canvas_len]
  * (the token each slot would receive); canvas: dev int32, in place;
