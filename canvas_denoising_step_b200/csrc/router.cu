@@ -34,27 +34,26 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
     float v[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = 0.f;
-    for (int s0 = 0; s0 < a.splits; s0 += 8) {   // 8 splits' loads in flight at once
-      float4 buf[8][2];
+    // the two expert halves in turn (E <= 256), 16 splits' loads in flight at once;
+    // each logit sums its splits in split order
 #pragma unroll
-      for (int ss = 0; ss < 8; ++ss)
+    for (int hh = 0; hh < 2; ++hh) {
+      const int e0 = 128 * hh + 4 * lane;
+      if (128 * hh >= E) break;
+      for (int s0 = 0; s0 < a.splits; s0 += 16) {
+        float4 buf[16];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int e0 = 128 * hh + 4 * lane;
+        for (int ss = 0; ss < 16; ++ss)
           if (s0 + ss < a.splits && e0 < E)
-            buf[ss][hh] = __ldg(reinterpret_cast<const float4*>(
+            buf[ss] = __ldg(reinterpret_cast<const float4*>(
                 a.logits_in + ((size_t)(s0 + ss) * T + t) * E + e0));
-        }
 #pragma unroll
-      for (int ss = 0; ss < 8; ++ss)
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int e0 = 128 * hh + 4 * lane;
+        for (int ss = 0; ss < 16; ++ss)
           if (s0 + ss < a.splits && e0 < E) {
-            v[4 * hh + 0] += buf[ss][hh].x; v[4 * hh + 1] += buf[ss][hh].y;
-            v[4 * hh + 2] += buf[ss][hh].z; v[4 * hh + 3] += buf[ss][hh].w;
+            v[4 * hh + 0] += buf[ss].x; v[4 * hh + 1] += buf[ss].y;
+            v[4 * hh + 2] += buf[ss].z; v[4 * hh + 3] += buf[ss].w;
           }
-        }
+      }
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {

@@ -338,7 +338,19 @@ __global__ void moe_gather_kernel(bf16* xperm, const int32_t* perm, int T, int k
   const int t = perm[p] / k;
   const uint4* src = reinterpret_cast<const uint4*>(xperm + (size_t)t * d);
   uint4* dst = reinterpret_cast<uint4*>(xperm + ((size_t)T + p) * d);
-  for (int i = threadIdx.x; i < d / 8; i += blockDim.x) dst[i] = src[i];
+  // all of this thread's 16-byte pieces are loaded before any is stored
+  constexpr int kPieces = 4;   // d / 8 <= 4 * 128 (d <= 4096)
+  uint4 r[kPieces];
+#pragma unroll
+  for (int u = 0; u < kPieces; ++u) {
+    const int i = threadIdx.x + (int)blockDim.x * u;
+    if (i < d / 8) r[u] = src[i];
+  }
+#pragma unroll
+  for (int u = 0; u < kPieces; ++u) {
+    const int i = threadIdx.x + (int)blockDim.x * u;
+    if (i < d / 8) dst[i] = r[u];
+  }
 }
 
 cudaError_t launch_moe_gather(bf16* xperm, const int32_t* perm, int T, int k, int d,
