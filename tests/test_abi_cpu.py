@@ -92,3 +92,17 @@ def test_null_arguments_and_no_device(dg):
         assert dg.raw_call(name, *args) == dg.DG_ERR_INVALID_ARG, name
     dg.dg_destroy(None)
     assert dg.dg_device_bytes(None) == 0
+
+
+def test_static_router_limits_checked_before_device_use(dg):
+    # argument errors are reported before any CUDA call, so no GPU is needed
+    p = 0x10000   # 16-byte aligned, never dereferenced
+    bad = [(0, 128, 8), (2049, 128, 8), (16, 2, 1), (16, 130, 8), (16, 260, 8), (16, 128, 0),
+           (16, 128, 9), (16, 4, 5)]
+    for rows, E, k in bad:
+        assert dg.raw_call("dg_router_topk_static", p, rows, E, k, p, p, p, p, None) == \
+            dg.DG_ERR_INVALID_ARG, (rows, E, k)
+    assert dg.raw_call("dg_router_topk_static", p + 4, 16, 128, 8, p, p, p, p, None) == \
+        dg.DG_ERR_INVALID_ARG
+    assert dg.raw_call("dg_router_topk_static", None, 16, 128, 8, p, p, p, p, None) == \
+        dg.DG_ERR_INVALID_ARG
