@@ -58,6 +58,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 _SIGS = {
     "dg_create": (c_int, [POINTER(DgConfig), c_void_p, POINTER(c_void_p)]),
     "dg_init_weights": (c_int, [c_void_p, c_uint64]),
+    "dg_load_weights": (c_int, [c_void_p, c_char_p, c_void_p, c_size_t]),
     "dg_set_prompt_kv": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_int, c_int]),
     "dg_set_router_bias": (c_int, [c_void_p, c_void_p]),
     "dg_canvas_step": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p]),
@@ -115,6 +116,10 @@ def dg_create(cfg: DgConfig, stream: int = 0) -> int:
 
 def dg_init_weights(ctx: int, seed: int) -> None:
     _check(ctx, _lib.dg_init_weights(ctx, seed), "dg_init_weights")
+
+
+def dg_load_weights(ctx: int, name: str, src: int, nbytes: int) -> None:
+    _check(ctx, _lib.dg_load_weights(ctx, name.encode(), src, nbytes), "dg_load_weights")
 
 
 def dg_set_prompt_kv(ctx: int, layer: int, k: int, v: int, batch: int, n_prompt: int) -> None:

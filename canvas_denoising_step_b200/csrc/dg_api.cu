@@ -795,6 +795,57 @@ int dg_commit(dg_ctx* c, const float* conf, int32_t* canvas, int batch, int step
   return DG_OK;
 }
 
+int dg_load_weights(dg_ctx* c, const char* name, const void* src, size_t bytes) {
+  if (!c || !name || !src) return DG_ERR_INVALID_ARG;
+  if (!c->weights_ready) return fail(c, DG_ERR_BAD_STATE, "weights not initialised");
+  const dg_config& cf = c->cfg;
+  const size_t d = cf.d_model, E = cf.n_experts, F = cf.d_ff, V = cf.vocab;
+  const size_t dh = cf.head_dim, Hq = cf.n_q_heads, Hkv = cf.n_kv_heads;
+  const std::string s(name);
+  // one contiguous destination, or rows of one bf16 matrix with a row pitch
+  void* dst = nullptr;
+  size_t n = 0, rows = 0, row_bytes = 0, pitch = 0;
+  if (s == "embed") { dst = c->embed; n = V * d * 2; }
+  else if (s == "ln_final") { dst = c->ln_final; n = d * 4; }
+  else {
+    const size_t colon = s.find(':');
+    if (colon == std::string::npos) return fail(c, DG_ERR_INVALID_ARG, "unknown tensor name");
+    const std::string base = s.substr(0, colon);
+    const int l = std::atoi(s.c_str() + colon + 1);
+    if (l < 0 || l >= cf.n_layers) return fail(c, DG_ERR_INVALID_ARG, "layer out of range");
+    Layer& L = c->layers[l];
+    bf16* gu = L.wgu;
+    if (base == "wq") { dst = L.wqkv; n = Hq * dh * d * 2; }
+    else if (base == "wk") { dst = L.wqkv + Hq * dh * d; n = Hkv * dh * d * 2; }
+    else if (base == "wv") { dst = L.wqkv + (Hq + Hkv) * dh * d; n = Hkv * dh * d * 2; }
+    else if (base == "wo") { dst = L.wo; n = d * Hq * dh * 2; }
+    else if (base == "wr") { dst = L.wr; n = E * d * 2; }
+    // gate/up rows are interleaved per group (row 2f gate, 2f + 1 up; group 0 shared):
+    // the (expert, f) rows of one kind are every second row from the group's first
+    else if (base == "wg") { dst = gu + 2 * F * d; rows = E * F; }
+    else if (base == "wu") { dst = gu + 2 * F * d + d; rows = E * F; }
+    else if (base == "sg") { dst = gu; rows = F; }
+    else if (base == "su") { dst = gu + d; rows = F; }
+    else if (base == "wd") { dst = L.wd + d * F; n = E * d * F * 2; }
+    else if (base == "sd") { dst = L.wd; n = d * F * 2; }
+    else if (base == "ln_in") { dst = L.ln_in; n = d * 4; }
+    else if (base == "ln_post") { dst = L.ln_post; n = d * 4; }
+    else if (base == "ln_ff") { dst = L.ln_ff; n = d * 4; }
+    else return fail(c, DG_ERR_INVALID_ARG, "unknown tensor name");
+    if ((base == "sg" || base == "su") && cf.n_shared == 0)
+      return fail(c, DG_ERR_INVALID_ARG, "the config has no shared expert");
+    if (rows) { row_bytes = d * 2; pitch = 2 * d * 2; n = rows * row_bytes; }
+  }
+  if (bytes != n) return fail(c, DG_ERR_INVALID_ARG, "byte count does not match the tensor");
+  if (rows)
+    DG_CUDA(c, cudaMemcpy2DAsync(dst, pitch, src, row_bytes, row_bytes, rows, cudaMemcpyDefault,
+                                 c->stream));
+  else
+    DG_CUDA(c, cudaMemcpyAsync(dst, src, n, cudaMemcpyDefault, c->stream));
+  DG_CUDA(c, cudaStreamSynchronize(c->stream));
+  return DG_OK;
+}
+
 int dg_debug_tensor(dg_ctx* c, const char* name, void* dst, size_t bytes, size_t* bytes_needed) {
   if (!c || !name) return DG_ERR_INVALID_ARG;
   const dg_config& cf = c->cfg;

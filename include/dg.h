@@ -103,6 +103,23 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out);
  * (seed, tensor, element index), never on the physical layout. */
 int dg_init_weights(dg_ctx* ctx, uint64_t seed);
 
+/* Replace one weight tensor with the caller's values, after dg_init_weights
+ * (which sets every tensor).  src: bf16 row-major of the logical shape below
+ * (fp32 for the norm weights), host or device memory, read during the call;
+ * bytes must equal the tensor's size exactly.  Names:
+ *   "embed" [vocab][d_model] (tied with the head), "ln_final" fp32 [d_model];
+ *   per layer l (the name carries ":l", e.g. "wq:3"):
+ *   "wq" [n_q_heads*head_dim][d_model], "wk" / "wv" [n_kv_heads*head_dim][d_model],
+ *   "wo" [d_model][n_q_heads*head_dim], "wr" [n_experts][d_model],
+ *   "wg" / "wu" [n_experts][d_ff][d_model] (routed gate / up), "wd" [n_experts][d_model][d_ff],
+ *   "sg" / "su" [d_ff][d_model], "sd" [d_model][d_ff] (the shared expert),
+ *   "ln_in" / "ln_post" / "ln_ff" fp32 [d_model].
+ * The values are copied into the library's own layout (q/k/v rows fused, gate
+ * and up rows interleaved).  Captured passes stay valid.  Returns DG_OK,
+ * DG_ERR_INVALID_ARG (unknown name, layer out of range, wrong size),
+ * DG_ERR_BAD_STATE (weights not initialised) or DG_ERR_CUDA. */
+int dg_load_weights(dg_ctx* ctx, const char* name, const void* src, size_t bytes);
+
 /* Borrows the prompt's cached keys and values for one layer (the encoder's KV
  * cache the decoder cross-attends to).  k, v: dev bf16 [batch][n_kv_heads]
  * [n_prompt][head_dim], keys already rotated.  No copy is made: the buffers

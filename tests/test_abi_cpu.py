@@ -106,3 +106,7 @@ def test_static_router_limits_checked_before_device_use(dg):
         dg.DG_ERR_INVALID_ARG
     assert dg.raw_call("dg_router_topk_static", None, 16, 128, 8, p, p, p, p, None) == \
         dg.DG_ERR_INVALID_ARG
+
+
+def test_load_weights_needs_a_context(dg):
+    assert dg.raw_call("dg_load_weights", None, b"wq:0", 0x10000, 16) == dg.DG_ERR_INVALID_ARG
