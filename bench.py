@@ -33,6 +33,7 @@ import sys
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
+METRIC = "canvas tokens/sec on 1 B200 (fixed denoise steps); % of HBM roofline per step"
 sys.path.insert(0, ROOT)
 
 WORKLOAD = "stack"
@@ -285,7 +286,7 @@ def run_reference(args, cfg, rank, world):
     t_step = statistics.mean(per)
     value = cfg["batch"] * cfg["canvas_len"] / (cfg["steps"] * t_step)
     unit = "canvas tokens/s"
-    line = {"metric": "canvas tokens/sec on 1 B200 (fixed denoise steps)", "value": value,
+    line = {"metric": METRIC, "value": value,
             "unit": unit, "impl": "reference", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -419,7 +420,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     step_ms = t_max / args.steps
     total_prof = sum(v[0] for v in kern.values())
     line = {
-        "metric": "canvas tokens/sec on 1 B200 (fixed denoise steps); % of HBM roofline per step",
+        "metric": METRIC,
         "value": value, "unit": "canvas tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
