@@ -18,6 +18,8 @@ numpy float64.  Each function cites the passage of the pages it follows:
   section "How Text Diffusion Actually Works".
 
 Where those pages are silent the reading taken is stated at the function.
+``eb_sampler`` holds the entropy-bounded denoising rule (the next row of the
+build; its readings are stated in that module).
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (brute force, closed forms, identities and invariants); the end-to-end values
 of a whole step are pinned only through those parts, because the pages print

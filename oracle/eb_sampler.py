@@ -1,0 +1,101 @@
+"""Entropy-bounded denoising (the next step after the fixed-step commit), CPU oracle.
+
+TEST INFRASTRUCTURE ONLY (see the package header): nothing on the product path
+imports this module.
+
+The pages name the sampler and its settings but not its steps:
+"DiffusionGemma: The Diffusion Era Begins with 4x Faster Text Generation"
+(efeozkan.com.tr), section "Recommended Inference Settings" -- an entropy-bound
+sampler, at most 48 denoising steps, a temperature that decays linearly from
+0.8 to 0.4, an entropy bound of 0.1, and an adaptive stop once the average canvas
+entropy is below 0.005 and the high-probability tokens have stayed the same for
+2 consecutive steps; "DiffusionGemma: Exploring the Paradigm Shift in
+Non-Autoregressive Language Modeling" (techsurvey.info), section "Serving in
+Production", repeats the 0.005 halting threshold.  The readings taken (E1-E5)
+are stated at each function.  Random draws are inputs (uniforms u in [0, 1)).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+N_MAX_STEPS = 48
+T_START, T_END = 0.8, 0.4
+ENTROPY_BOUND = 0.1
+STOP_ENTROPY = 0.005
+STOP_STABLE_STEPS = 2
+
+
+def eb_temperature(step: int, n_max: int = N_MAX_STEPS, t_start: float = T_START,
+                   t_end: float = T_END) -> float:
+    """E1: the temperature of step 0 .. n_max-1 falls linearly from t_start to t_end."""
+    if not 0 <= step < n_max:
+        raise ValueError("step out of range")
+    if n_max == 1:
+        return t_start
+    return t_start + (t_end - t_start) * step / (n_max - 1)
+
+
+def eb_row_stats(logits: np.ndarray, mask_id: int, temperature: float):
+    """E2: per row, the distribution softmax(l / T) over the vocabulary without the
+    mask id (as in the fixed-step head), its entropy H = -sum p ln p (nats), and
+    the argmax token (lowest index on ties).  Returns (H, argmax, p)."""
+    z = np.array(logits, dtype=np.float64, copy=True) / temperature
+    z[:, mask_id] = -np.inf
+    a = np.argmax(z, axis=1).astype(np.int32)
+    z = z - z[np.arange(z.shape[0]), a][:, None]
+    e = np.exp(z)
+    s = e.sum(axis=1)
+    p = e / s[:, None]
+    zp = np.where(p > 0, z, 0.0) * p
+    H = np.log(s) - zp.sum(axis=1)
+    return H, a, p
+
+
+def eb_sample(p: np.ndarray, u: np.ndarray) -> np.ndarray:
+    """E3: token i of each row by inverse CDF: the first vocab index whose
+    cumulative probability (in index order) exceeds u_i."""
+    c = np.cumsum(p, axis=1)
+    tok = np.empty(p.shape[0], dtype=np.int32)
+    for r in range(p.shape[0]):
+        j = 0
+        while j < p.shape[1] - 1 and c[r, j] <= u[r] * c[r, -1]:
+            j += 1
+        while p[r, j] == 0 and j > 0:   # never land on a zero-probability token
+            j -= 1
+        tok[r] = j
+    return tok
+
+
+def eb_unmask(canvas: np.ndarray, H: np.ndarray, tok: np.ndarray, mask_id: int,
+              bound: float = ENTROPY_BOUND):
+    """E4: in each canvas, the masked slots in order of entropy (lowest first, then
+    lowest slot) are committed while their summed entropy stays within the bound;
+    at least one slot is committed while any is masked.  canvas, tok int [B, Tc];
+    H [B, Tc].  Returns (new_canvas, committed bool [B, Tc])."""
+    canvas = np.array(canvas, dtype=np.int32, copy=True)
+    committed = np.zeros(canvas.shape, dtype=bool)
+    for b in range(canvas.shape[0]):
+        masked = [i for i in range(canvas.shape[1]) if canvas[b, i] == mask_id]
+        order = sorted(masked, key=lambda i: (float(H[b, i]), i))
+        total = 0.0
+        for n, i in enumerate(order):
+            total += float(H[b, i])
+            if n > 0 and total > bound:
+                break
+            canvas[b, i] = tok[b, i]
+            committed[b, i] = True
+    return canvas, committed
+
+
+def eb_should_stop(mean_entropy_history, argmax_history, threshold: float = STOP_ENTROPY,
+                   stable: int = STOP_STABLE_STEPS) -> bool:
+    """E5: stop once the canvas's mean entropy (over all its slots) at the latest step
+    is below the threshold and the argmax tokens of every slot have not changed
+    over the last `stable` steps (the latest `stable + 1` argmax vectors agree)."""
+    if len(mean_entropy_history) == 0 or mean_entropy_history[-1] >= threshold:
+        return False
+    if len(argmax_history) < stable + 1:
+        return False
+    last = [np.asarray(a) for a in argmax_history[-(stable + 1):]]
+    return all(np.array_equal(last[0], x) for x in last[1:])
