@@ -144,11 +144,13 @@ int dg_set_router_bias(dg_ctx* ctx, const float* bias);
  * committed_out (dev uint8 [batch][canvas_len]) receives 1 for the slots
  * committed by this pass.  Both may be NULL.
  * The pass is enqueued on the context's stream and the call returns without
- * waiting (dg_sync waits and reports device errors).  The second call for a
- * given batch records the pass into a CUDA graph that later calls replay;
- * dg_set_prompt_kv with other buffers or shapes, and dg_set_router_bias, drop
- * the recorded graphs.  Kernels are chained with programmatic dependent launch.
- * Setting DG_NO_GRAPH=1 or DG_NO_PDL=1 in the environment turns either off. */
+ * waiting (dg_sync waits and reports device errors).  On a context created
+ * with its own (non-default) stream and with profiling off, the second call
+ * for a given batch records the pass into a CUDA graph that later calls
+ * replay; dg_set_prompt_kv with other buffers or shapes, and
+ * dg_set_router_bias, drop the recorded graphs.  Kernels are chained with
+ * programmatic dependent launch.  Setting DG_NO_GRAPH=1 or DG_NO_PDL=1 in the
+ * environment turns either off. */
 int dg_canvas_step(dg_ctx* ctx, int32_t* canvas, int batch, int steps_left,
                    float* conf_out, uint8_t* committed_out);
 
