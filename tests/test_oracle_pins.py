@@ -423,3 +423,116 @@ def test_c_generator_matches_numpy_generator():
         a = orng.weight_tensor_numpy(0, tid, shape, 0.02, bf16, start=start)
         b = orng.weight_tensor(0, tid, shape, 0.02, bf16, start=start)
         assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+# ----------------------------------------------------------------------------- layer assembly
+
+def _wiring_cfg(**kw):
+    """d = dh = 4, one query and one key/value head, layer 0 local (window 1),
+    layer 1 global (p-RoPE with p = 0.25 rotates pair 0 only)."""
+    base = dict(n_layers=2, d_model=4, n_q_heads=1, n_kv_heads=1, head_dim=4, n_experts=2,
+                top_k=1, n_shared=0, d_ff=4, vocab=8, canvas_len=2, window=1, global_every=2,
+                rope_theta=10000.0, prope_fraction=0.25)
+    base.update(kw)
+    return om.OracleConfig(**base)
+
+
+def _wiring_weights(cfg, layer):
+    """Hand-set projections on h = e0 (input norm gives x = 2 e0): q = e0, canvas keys
+    0, canvas values e0, every other weight zero (the block adds nothing to h)."""
+    z = np.zeros((4, 4))
+    wq = z.copy(); wq[0, 0] = 0.5
+    wv = z.copy(); wv[0, 0] = 0.5
+    zero_expert = (np.zeros((4, 4)), np.zeros((4, 4)), np.zeros((4, 4)))
+    return _FixedWeights(cfg, layer, {"wq": wq, "wk": z.copy(), "wv": wv, "wo": z.copy(),
+                                      "wr": np.zeros((2, 4))}, [zero_expert] * 2)
+
+
+def _wiring_prompt(a=(1.0, -2.0, 4.0)):
+    """Three prompt keys a_j e0 and values (j + 1) e1, [B=1, Hkv=1, P=3, dh=4]."""
+    kp = np.zeros((1, 1, 3, 4))
+    vp = np.zeros((1, 1, 3, 4))
+    for j, aj in enumerate(a):
+        kp[0, 0, j, 0] = aj
+        vp[0, 0, j, 1] = j + 1
+    return kp, vp
+
+
+def _hand_attention(pos, a_visible, v_index):
+    """o at one canvas query, worked by hand: the rotated query at position `pos` is
+    (cos pos, 0, sin pos, 0) (pair 0 turns at frequency theta^0 = 1), so prompt key
+    a_j e0 scores a_j cos(pos) / sqrt(4); both canvas keys are 0 (score 0) and carry
+    the value e0; prompt value j is (j + 1) e1."""
+    e_p = [math.exp(aj * math.cos(pos) / 2.0) for aj in a_visible]
+    z = sum(e_p) + 2.0
+    return np.array([2.0 / z, sum(e * (j + 1) for e, j in zip(e_p, v_index)) / z, 0.0, 0.0])
+
+
+def test_layer_canvas_positions_window_and_unrotated_values():
+    """Canvas slot i attends from position P + i; a local layer sees only the last
+    min(window, P) prompt keys and a global one all P; V is never rotated
+    ("Hands-On with Diffusion Gemma", Detailed Specs: sliding-window local layers,
+    global layers, RoPE / p-RoPE; the readings R2 and R4)."""
+    cfg = _wiring_cfg()
+    a = (1.0, -2.0, 4.0)
+    kp, vp = _wiring_prompt(a)
+    h = np.zeros((1, 2, 4))
+    h[..., 0] = 1.0
+    P = 3
+    for layer, vis in ((0, [2]), (1, [0, 1, 2])):      # window 1 on the local layer
+        tr = {}
+        out = om.layer_forward(cfg, _wiring_weights(cfg, layer), h, kp, vp, trace=tr)
+        assert np.array_equal(out, h)                   # zero o-projection and experts
+        for i in range(2):
+            want = _hand_attention(P + i, [a[j] for j in vis], vis)
+            assert np.allclose(tr["attn_o"][0, i, 0], want, atol=1e-12), (layer, i)
+    # keys outside the window do not matter on the local layer, and do on the global one
+    kp2 = kp.copy()
+    kp2[0, 0, :2, 0] = (7.0, 3.0)
+    for layer, same in ((0, True), (1, False)):
+        t1, t2 = {}, {}
+        om.layer_forward(cfg, _wiring_weights(cfg, layer), h, kp, vp, trace=t1)
+        om.layer_forward(cfg, _wiring_weights(cfg, layer), h, kp2, vp, trace=t2)
+        assert np.array_equal(t1["attn_o"], t2["attn_o"]) == same, layer
+
+
+def test_layer_window_longer_than_prompt_sees_every_key():
+    """A window of 1024 over a 3-key prompt: the local layer sees all 3 (min(window, P))."""
+    cfg = _wiring_cfg(window=1024)
+    a = (1.0, -2.0, 4.0)
+    kp, vp = _wiring_prompt(a)
+    h = np.zeros((1, 2, 4))
+    h[..., 0] = 1.0
+    tr = {}
+    om.layer_forward(cfg, _wiring_weights(cfg, 0), h, kp, vp, trace=tr)
+    for i in range(2):
+        assert np.allclose(tr["attn_o"][0, i, 0], _hand_attention(3 + i, a, [0, 1, 2]),
+                           atol=1e-12)
+
+
+def test_canvas_step_final_norm_and_embedding_row(monkeypatch):
+    """A pass through identity blocks: the head scores the final-normed embedding row
+    of the mask id against the tied embedding, mask id excluded ("Hands-On with
+    Diffusion Gemma", Detailed Specs: tied embed_tokens / lm_head and the final norm).
+    Embedding (vocab 4, d 2, mask id 0): rows (1, 1), (2, 0), (0, 1.5), (-1, 2).
+    The canvas is all mask, so h = (1, 1); rms = 1, so the final norm leaves
+    (1, 1) / sqrt(1 + eps).  Logits of tokens 1..3: 2, 1.5, 1 (over sqrt(1 + eps)):
+    argmax 1 and confidence 1 / (1 + e^-0.5 + e^-1)."""
+    emb = np.array([[1.0, 1.0], [2.0, 0.0], [0.0, 1.5], [-1.0, 2.0]])
+    monkeypatch.setattr(om, "embedding_rows", lambda cfg, rows: emb[np.asarray(rows).ravel()])
+    monkeypatch.setattr(om, "embedding_block", lambda cfg, v0, v1: emb[v0:v1])
+    cfg = om.OracleConfig(n_layers=1, d_model=2, n_q_heads=1, n_kv_heads=1, head_dim=2,
+                          n_experts=1, top_k=1, n_shared=0, d_ff=2, vocab=4, canvas_len=3,
+                          window=4, global_every=1, rms_eps=1e-6)
+    z = np.zeros((2, 2))
+    W = _FixedWeights(cfg, 0, {"wq": z, "wk": z, "wv": z, "wo": z, "wr": np.zeros((1, 2))},
+                      [(z, z, z)])
+    kp = np.zeros((1, 1, 2, 2))
+    canvas = np.zeros((1, 3), np.int32)
+    new, conf, tok, com = om.canvas_step(cfg, canvas, [kp], [kp], 3, weights=[W])
+    s = 1.0 / math.sqrt(1.0 + 1e-6)
+    want = 1.0 / (1.0 + math.exp(-0.5 * s) + math.exp(-1.0 * s))
+    assert np.all(tok == 1)
+    assert np.allclose(conf, want, rtol=1e-12)
+    # one slot of three commits (k = ceil(3 / 3)); equal confidences -> slot 0
+    assert new.tolist() == [[1, 0, 0]] and com.tolist() == [[True, False, False]]
