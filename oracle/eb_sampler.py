@@ -91,11 +91,19 @@ def eb_unmask(canvas: np.ndarray, H: np.ndarray, tok: np.ndarray, mask_id: int,
 def eb_should_stop(mean_entropy_history, argmax_history, threshold: float = STOP_ENTROPY,
                    stable: int = STOP_STABLE_STEPS) -> bool:
     """E5: stop once the canvas's mean entropy (over all its slots) at the latest step
-    is below the threshold and the argmax tokens of every slot have not changed
-    over the last `stable` steps (the latest `stable + 1` argmax vectors agree)."""
+    is below the threshold and the argmax tokens of every slot agree over the last
+    `stable` consecutive steps (the latest `stable` argmax vectors are equal).
+
+    The two pages word the stability test differently: "DiffusionGemma: The
+    Diffusion Era Begins with 4x Faster Text Generation", Recommended Inference
+    Settings, has the high-probability tokens stay the same for 2 consecutive
+    steps; "DiffusionGemma: Exploring the Paradigm Shift in Non-Autoregressive
+    Language Modeling", Serving in Production, halts a block once two consecutive
+    passes reach consensus.  The reading that fits both: two consecutive passes
+    (2 argmax vectors) agree, so a block can stop at the second pass."""
     if len(mean_entropy_history) == 0 or mean_entropy_history[-1] >= threshold:
         return False
-    if len(argmax_history) < stable + 1:
+    if len(argmax_history) < max(stable, 1):
         return False
-    last = [np.asarray(a) for a in argmax_history[-(stable + 1):]]
+    last = [np.asarray(a) for a in argmax_history[-stable:]]
     return all(np.array_equal(last[0], x) for x in last[1:])

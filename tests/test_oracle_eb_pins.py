@@ -81,8 +81,12 @@ def test_unmask_takes_the_entropy_bounded_prefix():
 
 def test_adaptive_stop_needs_low_entropy_and_stable_argmax():
     a, b = np.array([1, 2, 3]), np.array([1, 2, 4])
-    assert not eb.eb_should_stop([0.004], [a, a])               # only one stable step
-    assert eb.eb_should_stop([0.01, 0.004], [a, a, a])
+    assert not eb.eb_should_stop([0.004], [a])                  # one pass: no consensus yet
+    assert eb.eb_should_stop([0.01, 0.004], [a, a])             # two consecutive passes agree
     assert not eb.eb_should_stop([0.004, 0.006], [a, a, a])     # entropy not low enough
-    assert not eb.eb_should_stop([0.004], [a, b, b])            # changed two steps back
-    assert eb.eb_should_stop([0.004], [b, a, a, a])
+    assert not eb.eb_should_stop([0.004], [a, a, b])            # the latest pass changed
+    assert eb.eb_should_stop([0.004], [b, a, a])                # older changes do not matter
+    assert not eb.eb_should_stop([0.004], [a, b])
+    # with stable = 3 the latest three passes must agree
+    assert not eb.eb_should_stop([0.004], [b, a, a], stable=3)
+    assert eb.eb_should_stop([0.004], [a, a, a], stable=3)
