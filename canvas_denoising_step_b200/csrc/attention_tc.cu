@@ -361,13 +361,8 @@ namespace {
 template <int DH>
 cudaError_t launch_attn_tc_t(const AttnTcMaps& m, const AttnTcArgs& a, cudaStream_t s) {
   const size_t smem = AttnSmem<DH>::kBytes + 1024;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DH>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(attn_tc_kernel<DH>), (int)smem);
+  if (e != cudaSuccess) return e;
   const int group = a.Hq / a.Hkv;
   dim3 grid((group * a.Tc + kRows - 1) / kRows, a.n_chunks, a.B * a.Hkv);
   return launch_k(attn_tc_kernel<DH>, grid, dim3(kThreads), smem, s, m.q, m.kc, m.vc, m.kp, m.vp,

@@ -205,6 +205,11 @@ std::string check_config(const dg_config& c) {
   if (!(c.rms_eps >= 0.f) || !(c.rope_theta > 0.f)) return "rms_eps must be >= 0 and rope_theta > 0";
   if (!(c.prope_fraction >= 0.f && c.prope_fraction <= 1.f)) return "prope_fraction must be in [0, 1]";
   if (!(c.weight_std > 0.0)) return "weight_std must be > 0";
+  // the router groups all rows of a pass in one CTA's shared memory
+  if (router_smem_bytes(c.max_batch * c.canvas_len, c.n_experts) >
+      (size_t)router_max_smem_bytes())
+    return "max_batch * canvas_len rows with n_experts experts exceed the router's shared "
+           "memory (2 * n_experts * ceil(rows / 32) + 2 * n_experts + 1 words <= 200 KB)";
   return "";
 }
 

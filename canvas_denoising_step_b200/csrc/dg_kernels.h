@@ -5,6 +5,12 @@
 
 namespace dg {
 
+// Raises the dynamic shared-memory limit of `func` to `bytes` on the current
+// device.  The attribute belongs to the device, so this is done once per
+// (kernel, device) pair; the table is guarded by a mutex, so host threads
+// driving different devices may launch at the same time.
+cudaError_t ensure_smem_limit(const void* func, int bytes);
+
 enum GemmMode { GEMM_DENSE = 0, GEMM_GATEUP = 1, GEMM_DOWN = 2, GEMM_HEAD = 3 };
 
 struct GemmArgs {
@@ -169,6 +175,7 @@ struct RouterArgs {
   int* err;
 };
 size_t router_smem_bytes(int T, int E);
+int router_max_smem_bytes();   // launch_router refuses larger shared-memory plans
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t s);
 // xperm[T + p] = xperm[perm[p] / k] for p < k*T (rows [0, T) hold the normed input).
 cudaError_t launch_moe_gather(bf16* xperm, const int32_t* perm, int T, int k, int d,

@@ -611,13 +611,8 @@ size_t gemm_smem_bytes(const GemmArgs& a) {
 cudaError_t gemm_tc_launch(const CUtensorMap& mapA, const CUtensorMap& mapB,
                            const CUtensorMap& mapC, const GemmArgs& a, int grid,
                            cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemm_tc_kernel), kMaxSmem);
+  if (e != cudaSuccess) return e;
   if (gemm_smem_bytes(a) > (size_t)kMaxSmem) return cudaErrorInvalidValue;
   return launch_k(gemm_tc_kernel, dim3(grid), dim3(kThreads), gemm_smem_bytes(a), stream, mapA,
                   mapB, mapC, a);

@@ -16,6 +16,7 @@ namespace dg {
 namespace {
 constexpr int kRouterThreads = 256;
 constexpr int kRowsPerBlock = kRouterThreads / 32;
+constexpr int kRouterMaxSmem = 200 * 1024;   // the grouping's shared-memory limit
 }  // namespace
 
 __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
@@ -209,6 +210,8 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
   if (threadIdx.x == 0) *a.counter = 0;
 }
 
+int router_max_smem_bytes() { return kRouterMaxSmem; }
+
 size_t router_smem_bytes(int T, int E) {
   const int W = (T + 31) / 32;
   return (size_t)(2 * E * W + E + E + 1) * sizeof(int);
@@ -216,13 +219,9 @@ size_t router_smem_bytes(int T, int E) {
 
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t s) {
   const size_t smem = router_smem_bytes(a.T, a.E);
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         200 * 1024);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  if (smem > (size_t)kRouterMaxSmem) return cudaErrorInvalidValue;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(router_kernel), kRouterMaxSmem);
+  if (e != cudaSuccess) return e;
   return launch_k(router_kernel, dim3((a.T + kRowsPerBlock - 1) / kRowsPerBlock),
                   dim3(kRouterThreads), smem, s, a);
 }

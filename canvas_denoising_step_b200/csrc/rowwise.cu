@@ -8,6 +8,9 @@
 // are issued together before any of them is used, so a CTA keeps tens of KB in
 // flight instead of one dependent round trip per source row.
 #include <cstdlib>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "dg_kernels.h"
 
@@ -71,6 +74,21 @@ __device__ __forceinline__ void st8b(bf16* p, const float* v) {
 }
 
 }  // namespace
+
+cudaError_t ensure_smem_limit(const void* func, int bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> done;   // (kernel, device) -> bytes set
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = done.find({func, dev});
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  done[{func, dev}] = bytes;
+  return cudaSuccess;
+}
 
 bool pdl_enabled() {
   static int v = -1;

@@ -70,7 +70,9 @@ typedef struct dg_ctx dg_ctx;
  *   n_q_heads a multiple of n_kv_heads; 1 <= top_k <= min(n_experts, 32);
  *   n_experts a multiple of 4 in [4, 256]; (n_q_heads + 2 n_kv_heads) * head_dim <= 16384;
  *   n_shared in {0, 1}; 1 <= canvas_len <= 256; max_batch * canvas_len <= 4096;
- *   0 <= mask_id < vocab; window >= 1; global_every >= 1.
+ *   0 <= mask_id < vocab; window >= 1; global_every >= 1;
+ *   2 * n_experts * ceil(max_batch * canvas_len / 32) + 2 * n_experts + 1 <= 51200
+ *   (the router groups a pass's rows in one CTA's 200 KB of shared memory).
  * Layer l (0-based) is global iff (l + 1) % global_every == 0: it attends to
  * all prompt keys and rotates the first ceil(prope_fraction * head_dim / 2)
  * RoPE pairs.  Other layers attend to the last min(window, n_prompt) prompt
@@ -89,13 +91,18 @@ typedef struct dg_config {
                                 instead of allocating more than this many device bytes */
 } dg_config;
 
-/* Creates a context on the current CUDA device: checks the config, allocates
+/* Pages: "Hands-On with Diffusion Gemma", Detailed Specs (the block structure
+ * and sizes a config describes).
+ * Creates a context on the current CUDA device: checks the config, allocates
  * the weights (bf16) and the workspace, and records `cuda_stream`
  * (a cudaStream_t, NULL = legacy default stream).  Weights are not yet drawn.
  * *out is set only on success.  Synchronous. */
 int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out);
 
-/* Draws every weight on the device from `seed` (the tied embedding, and per
+/* Pages: "Hands-On with Diffusion Gemma", Detailed Specs (the tensors: tied
+ * embed_tokens / lm_head, q/k/v/o, router, experts, shared expert, norms); the
+ * pages give no weight values, so they are seeded and synthetic.
+ * Draws every weight on the device from `seed` (the tied embedding, and per
  * layer the q/k/v/o projections, router, routed experts' gate/up/down and the
  * shared expert's gate/up/down), N(0, weight_std) by the SplitMix64 counter
  * generator with a four-term Irwin-Hall normal, rounded to bf16; norm scales
@@ -103,7 +110,8 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out);
  * (seed, tensor, element index), never on the physical layout. */
 int dg_init_weights(dg_ctx* ctx, uint64_t seed);
 
-/* Replace one weight tensor with the caller's values, after dg_init_weights
+/* Pages: "Hands-On with Diffusion Gemma", Detailed Specs (the tensor names).
+ * Replace one weight tensor with the caller's values, after dg_init_weights
  * (which sets every tensor).  src: bf16 row-major of the logical shape below
  * (fp32 for the norm weights), host or device memory, read during the call;
  * bytes must equal the tensor's size exactly.  Names:
@@ -120,7 +128,11 @@ int dg_init_weights(dg_ctx* ctx, uint64_t seed);
  * DG_ERR_BAD_STATE (weights not initialised) or DG_ERR_CUDA. */
 int dg_load_weights(dg_ctx* ctx, const char* name, const void* src, size_t bytes);
 
-/* Borrows the prompt's cached keys and values for one layer (the encoder's KV
+/* Pages: "Hands-On with Diffusion Gemma", Detailed Specs (the encoder's KV cache
+ * is shared with the decoder); "DiffusionGemma: The Diffusion Era Begins ...",
+ * DiffusionGemma's Technical Architecture (cross-attention into the prompt's
+ * cached KV).
+ * Borrows the prompt's cached keys and values for one layer (the encoder's KV
  * cache the decoder cross-attends to).  k, v: dev bf16 [batch][n_kv_heads]
  * [n_prompt][head_dim], keys already rotated.  No copy is made: the buffers
  * must stay valid and unchanged until this layer's next dg_set_prompt_kv or
@@ -130,11 +142,17 @@ int dg_load_weights(dg_ctx* ctx, const char* name, const void* src, size_t bytes
 int dg_set_prompt_kv(dg_ctx* ctx, int layer, const void* k, const void* v,
                      int batch, int n_prompt);
 
-/* Adds a fixed bias (dev fp32 [n_experts]) to the router logits of every
+/* The pages have no counterpart: a workload control (skewed expert popularity).
+ * Adds a fixed bias (dev fp32 [n_experts]) to the router logits of every
  * layer, or removes it when bias == NULL.  The bias is copied. */
 int dg_set_router_bias(dg_ctx* ctx, const float* bias);
 
-/* One denoising pass over `batch` canvases, then the commit.
+/* Pages: "Hands-On with Diffusion Gemma", How Is This Different from Previous
+ * Models? (a canvas of masked slots refined by repeated passes; the probability
+ * distribution judges which tokens are final) and "DiffusionGemma: The
+ * Diffusion Era Begins ...", What is Diffusion ... (locked-in tokens become
+ * context for the rest).
+ * One denoising pass over `batch` canvases, then the commit.
  * canvas: dev int32 [batch][canvas_len], updated in place: with r the number
  * of slots equal to mask_id in a canvas, the k = ceil(r / steps_left) masked
  * slots of highest confidence (ties toward the lower slot) receive their
@@ -154,24 +172,35 @@ int dg_set_router_bias(dg_ctx* ctx, const float* bias);
 int dg_canvas_step(dg_ctx* ctx, int32_t* canvas, int batch, int steps_left,
                    float* conf_out, uint8_t* committed_out);
 
-/* dg_canvas_step on HOST buffers: copies the canvas to the device, runs the
+/* Pages: as dg_canvas_step.
+ * dg_canvas_step on HOST buffers: copies the canvas to the device, runs the
  * pass, copies canvas (and conf / committed when not NULL) back, and returns
  * after the results are in host memory (synchronous). */
 int dg_canvas_step_host(dg_ctx* ctx, int32_t* canvas_host, int batch, int steps_left,
                         float* conf_host, uint8_t* committed_host);
 
-/* n_steps passes with steps_left = n_steps, n_steps - 1, ..., 1: every masked
+/* Pages: "DiffusionGemma: Google's Experimental Diffusion LLM", How Text
+ * Diffusion Actually Works (a small, fixed number of passes per block).
+ * n_steps passes with steps_left = n_steps, n_steps - 1, ..., 1: every masked
  * slot is committed at the end.  canvas: dev int32 [batch][canvas_len], in
  * place.  Ends with a synchronisation and reports device errors. */
 int dg_denoise_block(dg_ctx* ctx, int32_t* canvas, int batch, int n_steps);
 
-/* One decoder block on given hidden states (no embedding, head or commit):
+/* Pages: "Hands-On with Diffusion Gemma", Detailed Specs (input, post-attention
+ * and pre-feedforward norms, attention, MoE) and "DiffusionGemma: The Diffusion
+ * Era Begins ...", DiffusionGemma's Technical Architecture (bidirectional
+ * attention over the canvas, cross-attention into the prompt KV, 8 of 128
+ * experts + 1 shared).
+ * One decoder block on given hidden states (no embedding, head or commit):
  * x_out = block(x_in) with x_in, x_out dev bf16 [n_rows][d_model],
  * n_rows = batch * canvas_len for the batch given to dg_set_prompt_kv.
  * x_in and x_out may be the same buffer. */
 int dg_layer_forward(dg_ctx* ctx, int layer, const void* x_in, void* x_out, int n_rows);
 
-/* Router test hook: top_k selection and grouping from given logits.
+/* Pages: "DiffusionGemma: The Diffusion Era Begins ...", DiffusionGemma's
+ * Technical Architecture (8 of 128 experts active) and "Hands-On with Diffusion
+ * Gemma", Detailed Specs (the router).
+ * Router test hook: top_k selection and grouping from given logits.
  * logits: dev fp32 [n_rows][n_experts] (used as given; the router bias is not
  * added).  Outputs (dev): idx int32 [n_rows][top_k], experts by decreasing
  * logit, equal logits toward the lower index; w fp32 [n_rows][top_k], the
@@ -202,12 +231,17 @@ int dg_router_topk(dg_ctx* ctx, const float* logits, int n_rows, int32_t* idx, f
  * the stream at the start of each call; calls share it, so calls that may
  * overlap on the GPU (other streams, other host threads) race and must be
  * serialised by the caller.  Returns DG_OK, DG_ERR_INVALID_ARG or
- * DG_ERR_CUDA; the results are ready when the stream reaches them. */
+ * DG_ERR_CUDA; the results are ready when the stream reaches them.  The call
+ * does not wait for the GPU, so it reports no device-side error: the kernel's
+ * own checks (an expert index out of range, a total other than n_rows * top_k)
+ * cannot fire for inputs that pass the limits above, and if they did, the
+ * scratch error word they set would not be read back. */
 int dg_router_topk_static(const float* logits, int n_rows, int n_experts, int top_k,
                           int32_t* idx, float* w, int32_t* offsets, int32_t* perm,
                           void* cuda_stream);
 
-/* Self-test of the bounded waits that every kernel of the library uses (the
+/* The pages have no counterpart: failure detection.
+ * Self-test of the bounded waits that every kernel of the library uses (the
  * device half of the failure detection): runs one CTA on cuda_stream (NULL =
  * legacy default stream) that waits on an mbarrier nothing arrives on.  The
  * wait gives up after its limit (2 s), records DG_ERR_TIMEOUT and the kernel
@@ -217,14 +251,16 @@ int dg_router_topk_static(const float* logits, int n_rows, int n_experts, int to
  * allocates (and frees) one int of device memory. */
 int dg_selftest_bounded_wait(void* cuda_stream);
 
-/* Commit test hook: the commit rule of dg_canvas_step on given confidences.
+/* Pages: as dg_canvas_step (the locking of confident tokens).
+ * Commit test hook: the commit rule of dg_canvas_step on given confidences.
  * conf: dev fp32 [batch][canvas_len]; cand_tok: dev int32 [batch][canvas_len]
  * (the token each slot would receive); canvas: dev int32, in place;
  * committed_out: dev uint8 or NULL. */
 int dg_commit(dg_ctx* ctx, const float* conf, int32_t* canvas, int batch, int steps_left,
               const int32_t* cand_tok, uint8_t* committed_out);
 
-/* Debug hook: copies an internal tensor of the most recent pass (or layer
+/* The pages have no counterpart (inspection for tests).
+ * Debug hook: copies an internal tensor of the most recent pass (or layer
  * call) into dst (dev or host, `bytes` long; cudaMemcpyDefault), synchronously.
  * *bytes_needed (may be NULL) receives the tensor's size; with dst == NULL
  * only the size is reported.  Names and contents:
@@ -252,7 +288,8 @@ int dg_commit(dg_ctx* ctx, const float* conf, int32_t* canvas, int batch, int st
 int dg_debug_tensor(dg_ctx* ctx, const char* name, void* dst, size_t bytes,
                     size_t* bytes_needed);
 
-/* Instrumentation: with on != 0, every kernel launched by the following
+/* The pages have no counterpart (measurement).
+ * Instrumentation: with on != 0, every kernel launched by the following
  * passes is bracketed by CUDA events recorded on the context's stream (this
  * adds two event records per launch); on == 0 stops recording.  Either call
  * synchronises the stream and clears earlier records. */

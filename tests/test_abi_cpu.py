@@ -69,6 +69,25 @@ def test_invalid_configs_rejected_before_device_use(dg):
         assert dg.dg_last_error(None) != ""
 
 
+def test_configs_whose_router_grouping_cannot_fit_are_rejected(dg):
+    """4096 rows x 256 experts (264 KB) and x 200 experts (206 KB) of grouping state
+    exceed the router's 200 KB of shared memory: dg_create refuses them up front;
+    4096 rows x 128 experts (133 KB) is accepted by the checks (and then stops at
+    the missing device)."""
+    import synth
+    base = synth.config("tiny", canvas_len=256)
+    for E, want_reject in ((256, True), (200, True), (128, False)):
+        cfg = dg.config_from_dict(dict(base, n_experts=E), max_batch=16)
+        out = ctypes.c_void_p()
+        rc = dg.raw_call("dg_create", ctypes.byref(cfg), None, ctypes.byref(out))
+        msg = dg.dg_last_error(None)
+        if want_reject:
+            assert rc == dg.DG_ERR_INVALID_ARG and "router" in msg, (E, rc, msg)
+        else:
+            assert "router" not in msg, (E, msg)
+        assert out.value is None
+
+
 def test_null_arguments_and_no_device(dg):
     import synth
     cfg = dg.config_from_dict(synth.config("tiny"))
