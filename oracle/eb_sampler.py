@@ -11,7 +11,7 @@ sampler, at most 48 denoising steps, a temperature that decays linearly from
 entropy is below 0.005 and the high-probability tokens have stayed the same for
 2 consecutive steps; "DiffusionGemma: Exploring the Paradigm Shift in
 Non-Autoregressive Language Modeling" (techsurvey.info), section "Serving in
-Production", repeats the 0.005 halting threshold.  The readings taken (E1-E5)
+Production", repeats the 0.005 halting threshold.  The readings taken (E1-E6)
 are stated at each function.  Random draws are inputs (uniforms u in [0, 1)).
 """
 
@@ -107,3 +107,75 @@ def eb_should_stop(mean_entropy_history, argmax_history, threshold: float = STOP
         return False
     last = [np.asarray(a) for a in argmax_history[-stable:]]
     return all(np.array_equal(last[0], x) for x in last[1:])
+
+
+def eb_commit_step(canvas: np.ndarray, H: np.ndarray, argmax: np.ndarray, drawn: np.ndarray,
+                   prev_argmax, mask_id: int, last: bool, bound: float = ENTROPY_BOUND,
+                   threshold: float = STOP_ENTROPY):
+    """The decisions of one entropy-bounded pass, per canvas (E4, E5, E6).
+
+    canvas, argmax, drawn int [B, Tc]; H [B, Tc] (the pass's entropies);
+    prev_argmax int [B, Tc] or None (the previous pass's argmax tokens).
+    E5: a canvas stops when its mean entropy over all slots (summed in slot
+    order) is below the threshold and its argmax tokens equal the previous
+    pass's.  E6: a canvas that stops, or reaches the last allowed pass,
+    commits every still-masked slot with its argmax token; any other canvas
+    commits by the entropy bound (E4) with the drawn tokens.
+    Returns (new_canvas, committed bool [B, Tc], stopped bool [B])."""
+    canvas = np.array(canvas, dtype=np.int32, copy=True)
+    B, Tc = canvas.shape
+    committed = np.zeros((B, Tc), dtype=bool)
+    stopped = np.zeros(B, dtype=bool)
+    for b in range(B):
+        total = 0.0
+        for i in range(Tc):
+            total += float(H[b, i])
+        hist = [argmax[b]] if prev_argmax is None else [prev_argmax[b], argmax[b]]
+        stopped[b] = eb_should_stop([total / Tc], hist, threshold)
+        if stopped[b] or last:
+            for i in range(Tc):
+                if canvas[b, i] == mask_id:
+                    canvas[b, i] = argmax[b, i]
+                    committed[b, i] = True
+        else:
+            nb, cb = eb_unmask(canvas[b:b + 1], H[b:b + 1], drawn[b:b + 1], mask_id, bound)
+            canvas[b], committed[b] = nb[0], cb[0]
+    return canvas, committed, stopped
+
+
+def eb_denoise_block(cfg, canvas, k_prompt_layers, v_prompt_layers, u_steps,
+                     n_max: int = N_MAX_STEPS, weights=None, router_bias=None,
+                     history=None):
+    """Entropy-bounded denoising of one block of B canvases (E1-E6): pass s runs at
+    temperature eb_temperature(s, n_max), draws with the uniforms u_steps[s]
+    ([B, Tc]), and commits by eb_commit_step; a canvas that has stopped, or has no
+    masked slot left, is frozen while the others go on.  Ends when every canvas is
+    frozen or after n_max passes.  Returns (canvas, passes run per canvas)."""
+    from . import model as om
+    canvas = np.array(canvas, dtype=np.int32, copy=True)
+    B, Tc = canvas.shape
+    done = np.zeros(B, dtype=bool)
+    passes = np.zeros(B, dtype=np.int32)
+    prev = None
+    for s in range(n_max):
+        if done.all():
+            break
+        T = eb_temperature(s, n_max)
+        hn = om.final_hidden(cfg, canvas, k_prompt_layers, v_prompt_layers, router_bias, weights)
+        logits = hn @ om.embedding_block(cfg, 0, cfg.vocab).T
+        H, a, p = eb_row_stats(logits, cfg.mask_id, T)
+        drawn = eb_sample(p, np.asarray(u_steps[s]).reshape(-1))
+        H, a, drawn = H.reshape(B, Tc), a.reshape(B, Tc), drawn.reshape(B, Tc)
+        new, com, stop = eb_commit_step(canvas, H, a, drawn, prev, cfg.mask_id, s == n_max - 1)
+        for b in range(B):
+            if done[b]:
+                continue
+            canvas[b] = new[b]
+            passes[b] += 1
+            if stop[b] or not (canvas[b] == cfg.mask_id).any():
+                done[b] = True
+        if history is not None:
+            history.append(dict(canvas=canvas.copy(), H=H, argmax=a, drawn=drawn, committed=com,
+                                stopped=stop, done=done.copy()))
+        prev = a
+    return canvas, passes

@@ -412,6 +412,19 @@ def commit(canvas: np.ndarray, conf: np.ndarray, tok: np.ndarray, steps_left: in
     return canvas, committed
 
 
+def final_hidden(cfg: OracleConfig, canvas: np.ndarray, k_prompt_layers, v_prompt_layers,
+                 router_bias=None, weights=None) -> np.ndarray:
+    """The states the vocab head reads: embedding of the canvas tokens, every block,
+    then the final norm [HO Detailed Specs].  Returns hn [B * Tc, d]."""
+    c = cfg
+    B, Tc = canvas.shape
+    h = embedding_rows(c, canvas.reshape(-1)).reshape(B, Tc, c.d_model)
+    for layer in range(c.n_layers):
+        W = weights[layer] if weights is not None else layer_weights(c, layer)
+        h = layer_forward(c, W, h, k_prompt_layers[layer], v_prompt_layers[layer], router_bias)
+    return rmsnorm(h, np.ones(c.d_model), c.rms_eps).reshape(B * Tc, c.d_model)
+
+
 def canvas_step(cfg: OracleConfig, canvas: np.ndarray, k_prompt_layers, v_prompt_layers,
                 steps_left: int, router_bias=None, weights=None):
     """One denoising pass over the canvas, then the commit (R1-R14).
@@ -422,11 +435,7 @@ def canvas_step(cfg: OracleConfig, canvas: np.ndarray, k_prompt_layers, v_prompt
     """
     c = cfg
     B, Tc = canvas.shape
-    h = embedding_rows(c, canvas.reshape(-1)).reshape(B, Tc, c.d_model)
-    for layer in range(c.n_layers):
-        W = weights[layer] if weights is not None else layer_weights(c, layer)
-        h = layer_forward(c, W, h, k_prompt_layers[layer], v_prompt_layers[layer], router_bias)
-    hn = rmsnorm(h, np.ones(c.d_model), c.rms_eps).reshape(B * Tc, c.d_model)
+    hn = final_hidden(c, canvas, k_prompt_layers, v_prompt_layers, router_bias, weights)
     conf, tok, _, _ = head_reduce(c, hn)
     conf, tok = conf.reshape(B, Tc), tok.reshape(B, Tc)
     new_canvas, committed = commit(canvas, conf, tok, steps_left, c.mask_id)
