@@ -64,6 +64,11 @@ _SIGS = {
     "dg_canvas_step": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p]),
     "dg_canvas_step_host": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p]),
     "dg_denoise_block": (c_int, [c_void_p, c_void_p, c_int, c_int]),
+    "dg_eb_step": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
+                           c_void_p]),
+    "dg_eb_denoise_block": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p]),
+    "dg_eb_commit": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
+                             c_int, c_void_p, c_void_p]),
     "dg_layer_forward": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_int]),
     "dg_router_topk": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "dg_router_topk_static": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
@@ -144,6 +149,28 @@ def dg_canvas_step_host(ctx: int, canvas_host: int, batch: int, steps_left: int,
 
 def dg_denoise_block(ctx: int, canvas: int, batch: int, n_steps: int) -> None:
     _check(ctx, _lib.dg_denoise_block(ctx, canvas, batch, n_steps), "dg_denoise_block")
+
+
+def dg_eb_step(ctx: int, canvas: int, batch: int, step: int, n_max: int, u: int,
+               entropy_out: int | None = None, committed_out: int | None = None,
+               stopped_out: int | None = None) -> None:
+    _check(ctx, _lib.dg_eb_step(ctx, canvas, batch, step, n_max, u, entropy_out, committed_out,
+                                stopped_out), "dg_eb_step")
+
+
+def dg_eb_denoise_block(ctx: int, canvas: int, batch: int, n_max: int, u: int) -> list[int]:
+    """Runs the block; returns the passes each canvas took part in."""
+    passes = (c_int * batch)()
+    _check(ctx, _lib.dg_eb_denoise_block(ctx, canvas, batch, n_max, u, passes),
+           "dg_eb_denoise_block")
+    return list(passes)
+
+
+def dg_eb_commit(ctx: int, entropy: int, argmax: int, drawn: int, prev_argmax: int | None,
+                 canvas: int, batch: int, last: bool, committed_out: int | None = None,
+                 stopped_out: int | None = None) -> None:
+    _check(ctx, _lib.dg_eb_commit(ctx, entropy, argmax, drawn, prev_argmax, canvas, batch,
+                                  int(last), committed_out, stopped_out), "dg_eb_commit")
 
 
 def dg_layer_forward(ctx: int, layer: int, x_in: int, x_out: int, n_rows: int) -> None:

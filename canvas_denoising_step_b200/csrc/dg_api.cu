@@ -16,10 +16,22 @@ using namespace dg;
 
 namespace {
 
-constexpr int kGroupedTile = 128;   // B rows per grouped-GEMM tile
+#ifndef DG_GROUPED_TILE
+#define DG_GROUPED_TILE 256
+#endif
+constexpr int kGroupedTile = DG_GROUPED_TILE;   // rows of an expert chunk (B rows per grouped tile)
 constexpr int kGroupedBox = 32;     // B rows per TMA box of a grouped tile
+#ifndef DG_DOWN_PAIR
+#define DG_DOWN_PAIR 1
+#endif
+constexpr bool kDownPair = DG_DOWN_PAIR != 0;
 constexpr int kMaxAttnChunks = 16;
 constexpr int kMaxSplits = 16;
+// entropy-bounded denoising settings ("DiffusionGemma: The Diffusion Era Begins with
+// 4x Faster Text Generation", Recommended Inference Settings)
+constexpr double kEbBound = 0.1;          // entropy bound per pass (nats)
+constexpr double kEbStopEntropy = 0.005;  // mean canvas entropy that allows a stop
+constexpr double kEbTempStart = 0.8, kEbTempEnd = 0.4;
 
 std::string g_create_error;
 
@@ -67,6 +79,8 @@ struct dg_ctx {
   int* router_counter = nullptr;
   int* chunk_ready = nullptr;        // per-chunk gate/up -> down hand-over counters
   int n_chunk_ready = 0;
+  int32_t* chunk_order = nullptr;    // [n_chunk_ready] the expert chunks longest first
+  int* tile_counters = nullptr;      // [2] the gate/up and down GEMMs' dynamic tile counters
   int32_t *offsets_r = nullptr, *offsets_g = nullptr, *chunk_prefix = nullptr;
   int32_t *perm = nullptr, *inv = nullptr;
   bf16* H = nullptr;
@@ -74,6 +88,18 @@ struct dg_ctx {
   float *head_m = nullptr, *head_s = nullptr;
   int* head_a = nullptr;
   float* conf = nullptr;
+  float* head_max = nullptr;       // largest logit per row (mask id excluded)
+  // entropy-bounded passes
+  float* head_q = nullptr;         // [V/256][T] sum z e^z per vocab block
+  float* eb_H = nullptr;           // [T] entropy per row
+  float* eb_sum = nullptr;         // [T] sum e^((l - max) / temp)
+  float* eb_u = nullptr;           // [T] the pass's uniforms
+  int32_t* eb_prev = nullptr;      // [T] previous pass's argmax
+  int32_t* eb_drawn = nullptr;     // [T] drawn token of each committed slot
+  int* eb_state = nullptr;         // [Bmax] bit 0: eb_prev valid, bit 1: done
+  uint8_t* eb_stopped = nullptr;   // [Bmax]
+  float* eb_inv_temp = nullptr;    // 1 / temperature of the pass
+  int* eb_last = nullptr;          // the pass is the last allowed one
   int32_t* tok = nullptr;
   int32_t* canvas_dev = nullptr;
   uint8_t* committed_dev = nullptr;
@@ -92,7 +118,7 @@ struct dg_ctx {
   int last_T = 0, last_B = 0, launches = 0;
   int* steps_dev = nullptr;          // steps_left of the pass being run
   struct StepGraph { cudaGraphExec_t exec = nullptr; int launches = 0; };
-  std::map<int, StepGraph> graphs;   // captured passes, by batch size
+  std::map<int, StepGraph> graphs;   // captured passes, by 2 * batch size + (entropy-bounded)
   std::map<int, bool> warm;
   struct ProfRec { int kind; cudaEvent_t a, b; };
   bool prof_on = false;
@@ -261,7 +287,12 @@ int run_grouped(dg_ctx* c, int mode, const CUtensorMap& mA, const CUtensorMap& m
   a.M = M;
   a.n_tile = kGroupedTile;
   a.b_box_rows = kGroupedBox;
-  a.m_slabs = (M + 127) / 128;
+  // down: 256 weight rows per tile (its H chunk is read once per two slabs)
+  a.pair = mode == GEMM_DOWN && kDownPair ? 1 : 0;
+  a.m_slabs = a.pair ? (M + 255) / 256 : (M + 127) / 128;
+  a.chunk_order = c->chunk_order;
+  a.max_chunks = c->n_chunk_ready;
+  a.tile_counter = c->tile_counters + (mode == GEMM_DOWN ? 1 : 0);
   a.n_groups = cf.n_experts + 1;
   a.offsets = c->offsets_g;
   a.chunk_prefix = c->chunk_prefix;
@@ -336,6 +367,7 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
     ra.bitmap = c->bitmap; ra.counter = c->router_counter;
     ra.offsets_r = c->offsets_r; ra.offsets_g = c->offsets_g; ra.chunk_prefix = c->chunk_prefix;
     ra.chunk_ready = c->chunk_ready; ra.n_chunk_ready = c->n_chunk_ready;
+    ra.chunk_order = c->chunk_order; ra.tile_counters = c->tile_counters; ra.n_tile_counters = 2;
     ra.perm = c->perm; ra.inv = c->inv; ra.active_out = c->expert_active + l; ra.err = c->err_dev;
     DG_LAUNCH(c, K_ROUTER, launch_router(ra, c->stream));
   }
@@ -373,9 +405,12 @@ int ensure_rope(dg_ctx* c, int P) {
   return DG_OK;
 }
 
-// The kernels of one pass on c->canvas_dev (batch B): conf/tok into c->conf /
-// c->tok, commit in place with steps_left read from c->steps_dev.
-int record_step(dg_ctx* c, int B) {
+// The kernels of one pass on c->canvas_dev (batch B).  Fixed-step pass: conf/tok
+// into c->conf / c->tok, commit in place with steps_left read from c->steps_dev.
+// Entropy-bounded pass (eb): the head at temperature 1 / *c->eb_inv_temp, entropy
+// and argmax into c->eb_H / c->tok, then the stop test and the bounded commit
+// with the uniforms in c->eb_u.
+int record_step(dg_ctx* c, int B, bool eb) {
   const dg_config& cf = c->cfg;
   const int T = B * cf.canvas_len, d = cf.d_model;
   int rc;
@@ -396,15 +431,40 @@ int record_step(dg_ctx* c, int B) {
   a.n_vblocks = (cf.vocab + 255) / 256;
   a.n_tblocks = (T + 255) / 256;
   a.head_m = c->head_m; a.head_s = c->head_s; a.head_a = c->head_a;
+  if (eb) { a.inv_temp = c->eb_inv_temp; a.head_q = c->head_q; }
   a.err = c->err_dev;
   gemm_plan_smem(a);
   const int tiles = a.n_vblocks * a.n_tblocks;
   DG_LAUNCH(c, K_GEMM_HEAD, gemm_tc_launch(c->m_x_a, c->m_embed, c->m_Y_out, a,
                                            std::min(tiles, c->num_sms), c->stream));
-  DG_LAUNCH(c, K_HEAD_MERGE, launch_head_merge(c->head_m, c->head_s, c->head_a, a.n_vblocks, T, c->conf,
-                                 c->tok, c->stream));
-  DG_LAUNCH(c, K_COMMIT, launch_commit(c->conf, c->tok, c->canvas_dev, c->committed_dev, B, cf.canvas_len,
-                             -1, c->steps_dev, cf.mask_id, c->stream));
+  if (!eb) {
+    DG_LAUNCH(c, K_HEAD_MERGE, launch_head_merge(c->head_m, c->head_s, c->head_a, a.n_vblocks, T,
+                                                 c->conf, c->tok, c->head_max, c->stream));
+    DG_LAUNCH(c, K_COMMIT, launch_commit(c->conf, c->tok, c->canvas_dev, c->committed_dev, B,
+                                         cf.canvas_len, -1, c->steps_dev, cf.mask_id, c->stream));
+  } else {
+    EbMergeArgs m;
+    memset(&m, 0, sizeof(m));
+    m.T = T; m.n_vblocks = a.n_vblocks;
+    m.hm = c->head_m; m.hs = c->head_s; m.hq = c->head_q; m.ha = c->head_a;
+    m.inv_temp = c->eb_inv_temp;
+    m.H = c->eb_H; m.tok = c->tok; m.max_logit = c->head_max; m.sum = c->eb_sum;
+    DG_LAUNCH(c, K_HEAD_MERGE, launch_eb_merge(m, c->stream));
+    EbCommitArgs e;
+    memset(&e, 0, sizeof(e));
+    e.B = B; e.Tc = cf.canvas_len; e.T = T; e.mask_id = cf.mask_id; e.vocab = cf.vocab; e.d = d;
+    e.n_vblocks = a.n_vblocks;
+    e.H = c->eb_H; e.argmax = c->tok; e.u = c->eb_u; e.hn = c->x; e.embed = c->embed;
+    e.head_m = c->head_m; e.head_s = c->head_s; e.max_logit = c->head_max; e.sum = c->eb_sum;
+    e.inv_temp = c->eb_inv_temp;
+    e.prev_in = c->eb_prev; e.prev_out = c->eb_prev;
+    e.state = c->eb_state; e.state_out = c->eb_state;
+    e.last_flag = c->eb_last;
+    e.bound = kEbBound; e.threshold = kEbStopEntropy;
+    e.canvas = c->canvas_dev; e.committed = c->committed_dev; e.stopped = c->eb_stopped;
+    e.drawn_out = c->eb_drawn;
+    DG_LAUNCH(c, K_COMMIT, launch_eb_commit(e, c->stream));
+  }
   c->last_T = T;
   c->last_B = B;
   return DG_OK;
@@ -423,21 +483,22 @@ bool graphs_enabled(const dg_ctx* c) {
 }
 
 // One pass: the kernels run from a CUDA graph captured on the second pass of a
-// given batch size (the first runs directly and sets kernel attributes).
-int run_step(dg_ctx* c, int B, int steps_left) {
+// given (batch size, kind) (the first runs directly and sets kernel attributes).
+int run_step(dg_ctx* c, int B, int steps_left, bool eb = false) {
   int rc;
   if ((rc = ensure_rope(c, c->layers[0].kv_P)) != DG_OK) return rc;
-  DG_CUDA(c, launch_set_int(c->steps_dev, steps_left, c->stream));
-  if (!graphs_enabled(c)) return record_step(c, B);
-  auto it = c->graphs.find(B);
+  if (!eb) DG_CUDA(c, launch_set_int(c->steps_dev, steps_left, c->stream));
+  if (!graphs_enabled(c)) return record_step(c, B, eb);
+  const int key = 2 * B + (eb ? 1 : 0);
+  auto it = c->graphs.find(key);
   if (it == c->graphs.end()) {
-    if (!c->warm[B]) {
-      c->warm[B] = true;
-      return record_step(c, B);
+    if (!c->warm[key]) {
+      c->warm[key] = true;
+      return record_step(c, B, eb);
     }
     cudaGraph_t g = nullptr;
     DG_CUDA(c, cudaStreamBeginCapture(c->stream, cudaStreamCaptureModeThreadLocal));
-    rc = record_step(c, B);
+    rc = record_step(c, B, eb);
     const cudaError_t e = cudaStreamEndCapture(c->stream, &g);
     if (rc != DG_OK) {
       if (g) cudaGraphDestroy(g);
@@ -449,13 +510,36 @@ int run_step(dg_ctx* c, int B, int steps_left) {
     cudaGraphDestroy(g);
     if (e2 != cudaSuccess) return fail(c, DG_ERR_CUDA, std::string("graph instantiate: ") + cudaGetErrorString(e2));
     sg.launches = c->launches;
-    it = c->graphs.emplace(B, sg).first;
+    it = c->graphs.emplace(key, sg).first;
   }
   DG_CUDA(c, cudaGraphLaunch(it->second.exec, c->stream));
   c->launches = it->second.launches;
   c->last_T = B * c->cfg.canvas_len;
   c->last_B = B;
   return DG_OK;
+}
+
+// One entropy-bounded pass on c->canvas_dev: temperature and last-pass flag of
+// pass `step` of at most `n_max`, the uniforms copied into c->eb_u.
+int eb_pass(dg_ctx* c, int B, int step, int n_max, const float* u) {
+  const size_t T = (size_t)B * c->cfg.canvas_len;
+  const double temp = n_max == 1 ? kEbTempStart
+                                 : kEbTempStart + (kEbTempEnd - kEbTempStart) * step / (n_max - 1);
+  if (step == 0) DG_CUDA(c, cudaMemsetAsync(c->eb_state, 0, sizeof(int) * B, c->stream));
+  DG_CUDA(c, launch_set_float(c->eb_inv_temp, (float)(1.0 / temp), c->stream));
+  DG_CUDA(c, launch_set_int(c->eb_last, step == n_max - 1 ? 1 : 0, c->stream));
+  DG_CUDA(c, cudaMemcpyAsync(c->eb_u, u, T * 4, cudaMemcpyDefault, c->stream));
+  return run_step(c, B, 0, true);
+}
+
+int check_eb_args(dg_ctx* c, const void* canvas, int batch, const float* u, int n_max) {
+  if (!canvas || !u) return fail(c, DG_ERR_INVALID_ARG, "null canvas or uniforms");
+  if (batch < 1 || batch > c->cfg.max_batch) return fail(c, DG_ERR_INVALID_ARG, "batch out of range");
+  if (n_max < 1) return fail(c, DG_ERR_INVALID_ARG, "n_max must be >= 1");
+  if (!c->weights_ready) return fail(c, DG_ERR_BAD_STATE, "weights not initialised");
+  if (c->cfg.canvas_len > 256 || c->cfg.d_model % 8)
+    return fail(c, DG_ERR_UNSUPPORTED, "entropy-bounded passes need canvas_len <= 256");
+  return check_prompt_state(c, batch);
 }
 
 int read_device_error(dg_ctx* c) {
@@ -548,6 +632,8 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
     c->n_chunk_ready = (int)((T + kGroupedTile - 1) / kGroupedTile +
                              ((size_t)k * T + kGroupedTile - 1) / kGroupedTile + E);
     ok &= alloc_n(c, &c->chunk_ready, (size_t)c->n_chunk_ready);
+    ok &= alloc_n(c, &c->chunk_order, (size_t)c->n_chunk_ready);
+    ok &= alloc_n(c, &c->tile_counters, 2);
     ok &= alloc_n(c, &c->steps_dev, 4);
     ok &= alloc_n(c, &c->offsets_r, E + 1);
     ok &= alloc_n(c, &c->offsets_g, E + 2);
@@ -561,6 +647,17 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
     ok &= alloc_n(c, &c->head_s, nvb * T);
     ok &= alloc_n(c, &c->head_a, nvb * T);
     ok &= alloc_n(c, &c->conf, T);
+    ok &= alloc_n(c, &c->head_max, T);
+    ok &= alloc_n(c, &c->head_q, ((V + 255) / 256) * T);
+    ok &= alloc_n(c, &c->eb_H, T);
+    ok &= alloc_n(c, &c->eb_sum, T);
+    ok &= alloc_n(c, &c->eb_u, T);
+    ok &= alloc_n(c, &c->eb_prev, T);
+    ok &= alloc_n(c, &c->eb_drawn, T);
+    ok &= alloc_n(c, &c->eb_state, cf.max_batch);
+    ok &= alloc_n(c, &c->eb_stopped, cf.max_batch);
+    ok &= alloc_n(c, &c->eb_inv_temp, 4);
+    ok &= alloc_n(c, &c->eb_last, 4);
     ok &= alloc_n(c, &c->tok, T);
     ok &= alloc_n(c, &c->canvas_dev, T);
     ok &= alloc_n(c, &c->committed_dev, T);
@@ -582,7 +679,10 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
   cudaMemset(c->bitmap, 0, (size_t)E * ((T + 31) / 32) * 4);
   cudaMemset(c->router_counter, 0, 16);
   cudaMemset(c->chunk_ready, 0, sizeof(int) * (size_t)c->n_chunk_ready);
+  cudaMemset(c->chunk_order, 0, sizeof(int) * (size_t)c->n_chunk_ready);
+  cudaMemset(c->tile_counters, 0, sizeof(int) * 2);
   cudaMemset(c->err_dev, 0, 16);
+  cudaMemset(c->eb_state, 0, sizeof(int) * cf.max_batch);
   cudaMemset(c->expert_active, 0, sizeof(int) * cf.n_layers);
   cudaMemset(c->xperm, 0, rows_moe * d * 2);
   cudaMemset(c->H, 0, rows_moe * F * 2);
@@ -747,6 +847,67 @@ int dg_denoise_block(dg_ctx* c, int32_t* canvas, int batch, int n_steps) {
   return read_device_error(c);
 }
 
+int dg_eb_step(dg_ctx* c, int32_t* canvas, int batch, int step, int n_max, const float* u,
+               float* entropy_out, uint8_t* committed_out, uint8_t* stopped_out) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  int rc = check_eb_args(c, canvas, batch, u, n_max);
+  if (rc != DG_OK) return rc;
+  if (step < 0 || step >= n_max) return fail(c, DG_ERR_INVALID_ARG, "step must be in [0, n_max)");
+  const size_t T = (size_t)batch * c->cfg.canvas_len;
+  DG_CUDA(c, cudaMemcpyAsync(c->canvas_dev, canvas, T * 4, cudaMemcpyDefault, c->stream));
+  if ((rc = eb_pass(c, batch, step, n_max, u)) != DG_OK) return rc;
+  DG_CUDA(c, cudaMemcpyAsync(canvas, c->canvas_dev, T * 4, cudaMemcpyDefault, c->stream));
+  if (entropy_out)
+    DG_CUDA(c, cudaMemcpyAsync(entropy_out, c->eb_H, T * 4, cudaMemcpyDefault, c->stream));
+  if (committed_out)
+    DG_CUDA(c, cudaMemcpyAsync(committed_out, c->committed_dev, T, cudaMemcpyDefault, c->stream));
+  if (stopped_out)
+    DG_CUDA(c, cudaMemcpyAsync(stopped_out, c->eb_stopped, batch, cudaMemcpyDefault, c->stream));
+  return DG_OK;
+}
+
+int dg_eb_denoise_block(dg_ctx* c, int32_t* canvas, int batch, int n_max, const float* u,
+                        int* passes_out) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  int rc = check_eb_args(c, canvas, batch, u, n_max);
+  if (rc != DG_OK) return rc;
+  const size_t T = (size_t)batch * c->cfg.canvas_len;
+  std::vector<int> state(batch, 0), passes(batch, 0);
+  DG_CUDA(c, cudaMemcpyAsync(c->canvas_dev, canvas, T * 4, cudaMemcpyDefault, c->stream));
+  for (int s = 0; s < n_max; ++s) {
+    if ((rc = eb_pass(c, batch, s, n_max, u + (size_t)s * T)) != DG_OK) return rc;
+    for (int b = 0; b < batch; ++b) passes[b] += (state[b] & 2) ? 0 : 1;
+    DG_CUDA(c, cudaMemcpyAsync(state.data(), c->eb_state, sizeof(int) * batch,
+                               cudaMemcpyDeviceToHost, c->stream));
+    DG_CUDA(c, cudaStreamSynchronize(c->stream));
+    bool all_done = true;
+    for (int b = 0; b < batch; ++b) all_done = all_done && (state[b] & 2);
+    if (all_done) break;
+  }
+  DG_CUDA(c, cudaMemcpyAsync(canvas, c->canvas_dev, T * 4, cudaMemcpyDefault, c->stream));
+  if (passes_out) std::copy(passes.begin(), passes.end(), passes_out);
+  return read_device_error(c);
+}
+
+int dg_eb_commit(dg_ctx* c, const float* entropy, const int32_t* argmax, const int32_t* drawn,
+                 const int32_t* prev_argmax, int32_t* canvas, int batch, int last,
+                 uint8_t* committed_out, uint8_t* stopped_out) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (!entropy || !argmax || !drawn || !canvas) return fail(c, DG_ERR_INVALID_ARG, "null argument");
+  if (batch < 1 || batch > c->cfg.max_batch) return fail(c, DG_ERR_INVALID_ARG, "batch out of range");
+  if (c->cfg.canvas_len > 256) return fail(c, DG_ERR_UNSUPPORTED, "canvas_len must be <= 256");
+  EbCommitArgs e;
+  memset(&e, 0, sizeof(e));
+  e.B = batch; e.Tc = c->cfg.canvas_len; e.T = batch * c->cfg.canvas_len;
+  e.mask_id = c->cfg.mask_id; e.vocab = c->cfg.vocab; e.d = c->cfg.d_model;
+  e.H = entropy; e.argmax = argmax; e.drawn_in = drawn; e.prev_in = prev_argmax;
+  e.last = last ? 1 : 0;
+  e.bound = kEbBound; e.threshold = kEbStopEntropy;
+  e.canvas = canvas; e.committed = committed_out; e.stopped = stopped_out;
+  DG_CUDA(c, launch_eb_commit(e, c->stream));
+  return DG_OK;
+}
+
 int dg_layer_forward(dg_ctx* c, int layer, const void* x_in, void* x_out, int n_rows) {
   if (!c) return DG_ERR_INVALID_ARG;
   if (layer < 0 || layer >= c->cfg.n_layers) return fail(c, DG_ERR_INVALID_ARG, "layer out of range");
@@ -873,6 +1034,9 @@ int dg_debug_tensor(dg_ctx* c, const char* name, void* dst, size_t bytes, size_t
   else if (s == "perm") { src = c->perm; n = T * k * 4; }
   else if (s == "tok") { src = c->tok; n = T * 4; }
   else if (s == "conf") { src = c->conf; n = T * 4; }
+  else if (s == "head_max") { src = c->head_max; n = T * 4; }
+  else if (s == "entropy") { src = c->eb_H; n = T * 4; }
+  else if (s == "eb_drawn") { src = c->eb_drawn; n = T * 4; }
   else if (s == "embed") { src = c->embed; n = (size_t)cf.vocab * d * 2; }
   else if (s == "expert_active") { src = c->expert_active; n = (size_t)cf.n_layers * 4; }
   else {

@@ -31,6 +31,8 @@ struct GemmArgs {
   float* head_m;
   float* head_s;
   int* head_a;
+  const float* inv_temp;  // HEAD: NULL, or the inverse temperature (device) for the
+  float* head_q;          //   entropy variant, which also writes sum z e^z to head_q
   int* err;
   // shared-memory and TMEM plan (gemm_plan_smem)
   int stages, a_bytes, b_bytes, stage_bytes, b_box_rows;
@@ -41,6 +43,14 @@ struct GemmArgs {
   // once chunk_ready[c] reaches ready_target.  NULL: not used.
   int* chunk_ready;
   int ready_target;
+  // Grouped modes: tiles dealt longest chunk first from chunk_order (the router's
+  // order, max_chunks entries at most), taken one at a time from *tile_counter
+  // (zeroed by the router) when it is not NULL.  pair: a tile covers 256 weight
+  // rows (two accumulators; DOWN only).
+  const int* chunk_order;
+  int* tile_counter;
+  int max_chunks;
+  int pair;
   int tab_bytes;          // group tables in shared memory (grouped modes)
   int epi_bytes;          // fp32 output staging in shared memory (DENSE, DOWN)
 };
@@ -172,6 +182,9 @@ struct RouterArgs {
   int* active_out;         // += experts given rows, or NULL
   int* chunk_ready;        // [n_chunk_ready] set to 0 (the expert GEMMs' counters), or NULL
   int n_chunk_ready;
+  int32_t* chunk_order;    // [n_chunk_ready] chunks longest first (the GEMMs' tile order), or NULL
+  int* tile_counters;      // [n_tile_counters] set to 0 (the GEMMs' dynamic tile counters), or NULL
+  int n_tile_counters;
   int* err;
 };
 size_t router_smem_bytes(int T, int E);
@@ -186,9 +199,59 @@ cudaError_t launch_moe_combine(const float* Y, const float* w, const int32_t* in
                                int n_shared, int d, float* h, const float* w_next, float eps,
                                bf16* x, cudaStream_t s);
 
-// Vocab head merge over vocab blocks: conf = 1/sum, tok = argmax.
+// Vocab head merge over vocab blocks: conf = 1/sum, tok = argmax, max_logit = max.
 cudaError_t launch_head_merge(const float* hm, const float* hs, const int* ha, int n_vblocks,
-                              int T, float* conf, int32_t* tok, cudaStream_t s);
+                              int T, float* conf, int32_t* tok, float* max_logit,
+                              cudaStream_t s);
+// Entropy-bounded pass (eb_sampler.cu).  eb_merge folds the HEAD partials taken at
+// inverse temperature *inv_temp into per row: H (entropy, nats), tok (argmax),
+// max_logit and sum = sum_v e^((l_v - max) * inv_temp).
+struct EbMergeArgs {
+  int T, n_vblocks;
+  const float* hm;
+  const float* hs;
+  const float* hq;
+  const int* ha;
+  const float* inv_temp;
+  float* H;
+  int32_t* tok;
+  float* max_logit;
+  float* sum;
+};
+cudaError_t launch_eb_merge(const EbMergeArgs& a, cudaStream_t s);
+
+// One CTA per canvas: the stop test, then the commit at a stop / the last pass
+// (argmax tokens) or by the entropy bound (drawn tokens; drawn_in given: those
+// tokens, no draw).  state[b] (optional): bit 0 = prev_in holds the previous
+// pass's argmax, bit 1 = the canvas is done (left unchanged).
+struct EbCommitArgs {
+  int B, Tc, T, mask_id, vocab, d, n_vblocks;
+  const float* H;
+  const int32_t* argmax;
+  const int32_t* drawn_in;   // NULL: draw from the head partials
+  const float* u;            // [T] uniforms of the draw
+  const bf16* hn;            // [T][d] the states the head read
+  const bf16* embed;         // [vocab][d]
+  const float* head_m;       // [n_vblocks][T]
+  const float* head_s;
+  const float* max_logit;    // [T] (eb_merge)
+  const float* sum;          // [T]
+  const float* inv_temp;
+  const int32_t* prev_in;    // [T] previous argmax or NULL
+  const int* state;          // [B] or NULL
+  int32_t* prev_out;         // [T] or NULL
+  int* state_out;            // [B] or NULL
+  const int* last_flag;      // device flag "last allowed pass", or NULL: use `last`
+  int last;
+  double bound, threshold;
+  int32_t* canvas;
+  uint8_t* committed;        // [T] or NULL
+  uint8_t* stopped;          // [B] or NULL
+  int32_t* drawn_out;        // [T] or NULL: the drawn token of each committed slot
+};
+cudaError_t launch_eb_commit(const EbCommitArgs& a, cudaStream_t s);
+cudaError_t launch_set_float(float* p, float v, cudaStream_t s);
+
 // Commit (one block per canvas).  steps_left read from *steps_left_dev when
 // steps_left < 0.
 cudaError_t launch_commit(const float* conf, const int32_t* tok, int32_t* canvas,

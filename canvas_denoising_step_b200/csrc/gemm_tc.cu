@@ -25,7 +25,9 @@
 //  DOWN    Y[r][m] = sum_k H[r][k] Wd[g][m][k]                   (fp32)
 //  HEAD    per token row t and 256-wide vocab block b: the max logit, its
 //          index (lowest on ties) and sum exp(l - max) over the block, with
-//          the mask id and out-of-range vocab rows excluded      (partials)
+//          the mask id and out-of-range vocab rows excluded      (partials);
+//          with inv_temp set, the sums are taken of exp(z) and z exp(z) with
+//          z = (l - max) * inv_temp (the entropy of the block at that temperature)
 #include "dg_kernels.h"
 
 namespace dg {
@@ -40,6 +42,7 @@ constexpr int kMaxSmem = 232448;        // dynamic shared memory per CTA (227 KB
 
 struct TileInfo {
   int g, m_slab, row0, rows, kb0, kb1, split, tb, vb;
+  int chunk;   // grouped: the chunk (group-major numbering shared by GATEUP and DOWN)
   int a_row0;  // first A row of the tile (accumulator i covers a_row0 + 128 i ..)
   int n_acc;   // accumulators (A tiles) per tile
   int n_mma;   // MMA N
@@ -66,10 +69,11 @@ __device__ __forceinline__ int tile_count(const GemmArgs& a, const int* s_prefix
   }
 }
 
+// s_order: the chunks longest first (grouped modes with a chunk order), else NULL
 __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t, const int* s_prefix,
-                                               const int* s_offsets) {
+                                               const int* s_offsets, const int* s_order) {
   TileInfo ti;
-  ti.g = 0; ti.split = 0; ti.tb = 0; ti.vb = 0; ti.n_acc = 1;
+  ti.g = 0; ti.split = 0; ti.tb = 0; ti.vb = 0; ti.n_acc = 1; ti.chunk = 0;
   if (a.mode == GEMM_DENSE) {
     const int n_chunks = (a.N + a.n_tile - 1) / a.n_tile;
     ti.m_slab = t % a.m_slabs;
@@ -83,8 +87,12 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t, const 
     ti.n_acc = a.dense_pair ? 2 : 1;
     ti.a_row0 = ti.m_slab * 128 * ti.n_acc;
   } else if (a.mode == GEMM_GATEUP || a.mode == GEMM_DOWN) {
+    // tile t = (k-th chunk of the order, weight slab): all slabs of the longest
+    // chunk are dealt first; with `pair` a slab is 256 weight rows (two accumulators)
     ti.m_slab = t % a.m_slabs;
-    const int c = t / a.m_slabs;
+    const int k = t / a.m_slabs;
+    const int c = s_order ? s_order[k] : k;
+    ti.chunk = c;
     ti.g = upper_bound_prefix(s_prefix, a.n_groups, c);
     const int j = c - s_prefix[ti.g];
     const int beg = s_offsets[ti.g], end = s_offsets[ti.g + 1];
@@ -92,7 +100,8 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t, const 
     ti.rows = min(a.n_tile, end - ti.row0);
     ti.kb0 = 0;
     ti.kb1 = a.n_kb;
-    ti.a_row0 = ti.m_slab * 128;
+    ti.a_row0 = ti.m_slab * 128 * (a.pair ? 2 : 1);
+    ti.n_acc = (a.pair && ti.a_row0 + 128 < a.M) ? 2 : 1;
   } else {  // HEAD
     ti.tb = t % a.n_tblocks;
     ti.vb = t / a.n_tblocks;
@@ -120,8 +129,7 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
   return v;
 }
 
-// the chunk index of a grouped tile (the same numbering in GATEUP and DOWN)
-__device__ __forceinline__ int tile_chunk(const GemmArgs& a, int t) { return t / a.m_slabs; }
+constexpr int kTileQ = 4;   // depth of the dynamic tile queue (grouped modes)
 
 }  // namespace
 
@@ -133,15 +141,23 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                                              ~uintptr_t(1023));
   const int S = a.stages;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * a.stage_bytes);
-  // full[0..S), empty[S..2S), tmem_full[2S..2S+2), tmem_empty[2S+2..2S+4)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
+  // full[0..S), empty[S..2S), tmem_full[2S..2S+2), tmem_empty[2S+2..2S+4),
+  // tile queue full / empty [2S+4 .. 2S+4+2*kTileQ)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4 + 2 * kTileQ);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* s_tq = reinterpret_cast<volatile int*>(tmem_slot + 2);   // [kTileQ] tiles
   const uint32_t smem_base = smem_u32(smem);
   const uint32_t bar_base = smem_u32(bars);
   auto full_bar = [&](int s) { return bar_base + 8u * s; };
   auto empty_bar = [&](int s) { return bar_base + 8u * (S + s); };
   auto tfull_bar = [&](int b) { return bar_base + 8u * (2 * S + b); };
   auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * S + 2 + b); };
+  auto tq_full_bar = [&](int q) { return bar_base + 8u * (2 * S + 4 + q); };
+  auto tq_empty_bar = [&](int q) { return bar_base + 8u * (2 * S + 4 + kTileQ + q); };
+  // grouped modes with a tile counter deal tiles dynamically: the producer takes
+  // the next tile from the counter and passes it to the MMA and epilogue warps
+  // through a small queue; otherwise CTA b takes tiles b, b + grid, ...
+  const bool dyn = (a.mode == GEMM_GATEUP || a.mode == GEMM_DOWN) && a.tile_counter != nullptr;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -152,6 +168,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
       mbar_init(tempty_bar(b), 4);
+    }
+    for (int q = 0; q < kTileQ; ++q) {
+      mbar_init(tq_full_bar(q), 1);
+      mbar_init(tq_empty_bar(q), 5);   // the MMA lane and the four epilogue warps
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -175,6 +195,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   // launch: the tables are read before this kernel's wait.
   int* s_prefix = reinterpret_cast<int*>(smem + (size_t)S * a.stage_bytes + 1024);
   int* s_offsets = s_prefix + (a.n_groups + 1);
+  int* s_order = a.chunk_order ? s_offsets + (a.n_groups + 1) : nullptr;
   float* s_stage_out = reinterpret_cast<float*>(smem + (size_t)S * a.stage_bytes + 1024 + a.tab_bytes);
   const bool grouped = a.mode == GEMM_GATEUP || a.mode == GEMM_DOWN;
   if (grouped) {
@@ -183,13 +204,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       s_offsets[i] = __ldcg(a.offsets + i);
     }
     __syncthreads();
+    if (s_order)
+      for (int i = threadIdx.x; i < s_prefix[a.n_groups]; i += blockDim.x)
+        s_order[i] = __ldcg(a.chunk_order + i);
+    __syncthreads();
   }
   // The weights do not depend on the previous kernel either: the producer
   // issues the weight operand of its first tile's first stages now (fresh
   // barriers, no empty waits), and the activation operand after the wait.
   int pre = 0;
-  if (warp == 0 && lane == 0 && (int)blockIdx.x < tile_count(a, s_prefix)) {
-    const TileInfo ti = decode_tile(a, blockIdx.x, s_prefix, s_offsets);
+  int first_t = blockIdx.x;
+  // the first dynamic tile (the counter was zeroed by the router, which has
+  // completed, as the tables above)
+  if (dyn && warp == 0 && lane == 0) first_t = atomicAdd(a.tile_counter, 1);
+  if (warp == 0 && lane == 0 && first_t < tile_count(a, s_prefix)) {
+    const TileInfo ti = decode_tile(a, first_t, s_prefix, s_offsets, s_order);
     const uint32_t tx = (uint32_t)(ti.n_acc * kATileBytes) +
                         (uint32_t)(ti.n_bbox * a.b_box_rows * 128);
     pre = min(S, ti.kb1 - ti.kb0);
@@ -203,7 +232,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       } else if (a.mode == GEMM_HEAD) {
         tma_load_2d(sA + (uint32_t)a.a_bytes, &mapB, full_bar(p), kx, ti.row0);
       } else {
-        tma_load_3d(sA, &mapA, full_bar(p), kx, ti.a_row0, ti.g);
+        for (int i = 0; i < ti.n_acc; ++i)
+          tma_load_3d(sA + i * kATileBytes, &mapA, full_bar(p), kx, ti.a_row0 + i * 128, ti.g);
       }
     }
   }
@@ -226,14 +256,31 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       int stage = 0;
       uint32_t phase = 0;
       bool wrapped = false, ok = true;
-      bool first = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, first = false) {
-        const TileInfo ti = decode_tile(a, t, s_prefix, s_offsets);
+      for (int it = 0; ok; ++it) {
+        int t;
+        if (dyn) {
+          // take the next tile and publish it to the MMA and epilogue warps
+          const int q = it % kTileQ;
+          if (!mbar_wait(tq_empty_bar(q), (uint32_t)((it / kTileQ) & 1) ^ 1u, abort_flag, a.err)) {
+            ok = false;
+            break;
+          }
+          t = it == 0 ? first_t : atomicAdd(a.tile_counter, 1);
+          if (t >= n_tiles) t = -1;
+          s_tq[q] = t;
+          mbar_arrive(tq_full_bar(q));
+          if (t < 0) break;
+        } else {
+          t = blockIdx.x + it * gridDim.x;
+          if (t >= n_tiles) break;
+        }
+        const bool first = it == 0;
+        const TileInfo ti = decode_tile(a, t, s_prefix, s_offsets, s_order);
         const uint32_t tx = (uint32_t)(ti.n_acc * kATileBytes) +
                             (uint32_t)(ti.n_bbox * a.b_box_rows * 128);
         if (handover) {
           // this chunk's H rows are written by every gate/up slab's epilogue
-          const int* rc = a.chunk_ready + tile_chunk(a, t);
+          const int* rc = a.chunk_ready + ti.chunk;
           const unsigned long long t0 = globaltimer_ns();
           while (ld_acquire(rc) < a.ready_target) {
             if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
@@ -265,7 +312,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
             for (int i = 0; i < ti.n_acc; ++i)
               tma_load_2d(sA + i * kATileBytes, &mapA, fb, kx, ti.a_row0 + i * 128);
           } else if (!weight_issued) {
-            tma_load_3d(sA, &mapA, fb, kx, ti.a_row0, ti.g);
+            for (int i = 0; i < ti.n_acc; ++i)
+              tma_load_3d(sA + i * kATileBytes, &mapA, fb, kx, ti.a_row0 + i * 128, ti.g);
           }
           if (!(weight_issued && a.mode == GEMM_HEAD))
             for (int i = 0; i < ti.n_bbox; ++i)
@@ -288,9 +336,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int it = 0;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
-        const TileInfo ti = decode_tile(a, t, s_prefix, s_offsets);
+      for (int it = 0; ok; ++it) {
+        int t;
+        if (dyn) {
+          const int q = it % kTileQ;
+          if (!mbar_wait(tq_full_bar(q), (uint32_t)((it / kTileQ) & 1), abort_flag, a.err)) break;
+          t = s_tq[q];
+          mbar_arrive(tq_empty_bar(q));
+          if (t < 0) break;
+        } else {
+          t = blockIdx.x + it * gridDim.x;
+          if (t >= n_tiles) break;
+        }
+        const TileInfo ti = decode_tile(a, t, s_prefix, s_offsets, s_order);
         const int buf = it % n_bufs;
         const uint32_t tph = (uint32_t)((it / n_bufs) & 1);
         if (!mbar_wait(tempty_bar(buf), tph ^ 1u, abort_flag, a.err)) { ok = false; break; }
@@ -327,9 +385,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     const int n_sbuf = a.epi_bytes / (4 * 4096);
     float* s_warp_out = s_stage_out + (warp - 2) * n_sbuf * 1024;
     int sbuf = 0;
-    int it = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
-      const TileInfo ti = decode_tile(a, t, s_prefix, s_offsets);
+    for (int it = 0;; ++it) {
+      int t;
+      if (dyn) {
+        const int q = it % kTileQ;
+        if (!mbar_wait(tq_full_bar(q), (uint32_t)((it / kTileQ) & 1), abort_flag, a.err)) break;
+        t = s_tq[q];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tq_empty_bar(q));
+        if (t < 0) break;
+      } else {
+        t = blockIdx.x + it * gridDim.x;
+        if (t >= n_tiles) break;
+      }
+      const TileInfo ti = decode_tile(a, t, s_prefix, s_offsets, s_order);
       const int buf = it % n_bufs;
       const uint32_t tph = (uint32_t)((it / n_bufs) & 1);
       if (!mbar_wait(tfull_bar(buf), tph, abort_flag, a.err)) break;
@@ -377,7 +446,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
             }
           }
         }
-      } else if (a.mode == GEMM_GATEUP) {
+      } else if (a.mode == GEMM_GATEUP) {   // one 128-row slab per tile (no pair)
         // Interleaved rows: even accumulator rows are gate rows, odd rows the
         // matching up rows of the same output feature f.
         // A warp's 16 gate rows are 16 consecutive features f0 .. f0+15; a full
@@ -434,9 +503,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
           // this warp's H writes of the tile are visible before the count
           __threadfence();
           __syncwarp();
-          if (lane == 0) atomicAdd(a.chunk_ready + tile_chunk(a, t), 1);
+          if (lane == 0) atomicAdd(a.chunk_ready + ti.chunk, 1);
         }
-      } else {  // HEAD
+      } else if (a.inv_temp == nullptr) {  // HEAD
         for (int i = 0; i < ti.n_acc; ++i) {
           const int tok_row = ti.tb * 256 + i * 128 + r;
           float mx = -INFINITY, sum = 0.f;
@@ -464,6 +533,51 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
             a.head_m[o] = mx;
             a.head_s[o] = sum;
             a.head_a[o] = arg;
+          }
+        }
+      } else {  // HEAD with the entropy statistics at temperature 1 / inv_temp
+        // z = (l - mx) / temp; S = sum e^z; Q = sum z e^z; when the max grows by
+        // d = (mx_old - mx_new) / temp, S <- e^d S and Q <- e^d (Q + d S).
+        const float it = *a.inv_temp;
+        for (int i = 0; i < ti.n_acc; ++i) {
+          const int tok_row = ti.tb * 256 + i * 128 + r;
+          float mx = -INFINITY, sum = 0.f, qz = 0.f;
+          int arg = -1;
+          for (int c0 = 0; c0 < 256; c0 += 32) {
+            tmem_ld32(lane_addr + (uint32_t)i * kAccCols + (uint32_t)c0, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int vid = ti.row0 + c0 + j;
+              if (vid < a.vocab && vid != a.mask_id) {
+                const float x = __uint_as_float(v[j]);
+                if (x > mx) {
+                  if (arg < 0) {
+                    sum = 1.0f;
+                    qz = 0.f;
+                  } else {
+                    const float dz = (mx - x) * it;
+                    const float e = __expf(dz);
+                    qz = e * (qz + dz * sum);
+                    sum = e * sum + 1.0f;
+                  }
+                  mx = x;
+                  arg = vid;
+                } else {
+                  const float z = (x - mx) * it;
+                  const float e = __expf(z);
+                  sum += e;
+                  qz += z * e;
+                }
+              }
+            }
+          }
+          if (tok_row < a.T) {
+            const size_t o = (size_t)ti.vb * a.T + tok_row;
+            a.head_m[o] = mx;
+            a.head_s[o] = sum;
+            a.head_a[o] = arg;
+            a.head_q[o] = qz;
           }
         }
       }
@@ -582,12 +696,14 @@ bool make_tmap_f32_sw128(CUtensorMap* map, float* base, uint64_t inner, uint64_t
 // columns when a tile has one accumulator (so the epilogue of one tile
 // overlaps the MMAs of the next), one buffer of two when it has two.
 void gemm_plan_smem(GemmArgs& a) {
-  const int n_a = (a.mode == GEMM_HEAD || (a.mode == GEMM_DENSE && a.dense_pair)) ? 2 : 1;
+  const bool grouped = a.mode == GEMM_GATEUP || a.mode == GEMM_DOWN;
+  const int n_a = (a.mode == GEMM_HEAD || (a.mode == GEMM_DENSE && a.dense_pair) ||
+                   (grouped && a.pair)) ? 2 : 1;
   a.n_bufs = n_a == 1 ? 2 : 1;
   // group tables; fp32 output staging: two 4 KB blocks per epilogue warp for
   // DENSE, one for DOWN (which keeps its sixth operand stage)
-  a.tab_bytes = (a.mode == GEMM_GATEUP || a.mode == GEMM_DOWN)
-                    ? ((2 * (a.n_groups + 1) * 4 + 127) / 128) * 128 : 0;
+  a.tab_bytes = grouped ? ((2 * (a.n_groups + 1) * 4 + (a.chunk_order ? a.max_chunks * 4 : 0) +
+                            127) / 128) * 128 : 0;
   a.epi_bytes = a.mode == GEMM_DENSE ? 2 * 4 * 4096
                 : (a.mode == GEMM_DOWN ? 4 * 4096 : (a.mode == GEMM_GATEUP ? 2 * 4 * 1024 : 0));
   a.a_bytes = n_a * kATileBytes;

@@ -118,6 +118,10 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
   int* count = sm_dyn + E * W;   // [E]
   int* off = count + E;          // [E + 1]
   uint32_t* words = reinterpret_cast<uint32_t*>(off + E + 1);  // [E * W]
+  int* cpre = reinterpret_cast<int*>(words + E * W);   // [E + 2] chunk prefix of the groups
+  int* fbase = cpre + E + 2;                           // [E + 1] first order slot of a group's full chunks
+  int* prow = fbase + E + 1;                           // [E + 1] rows of a group's partial chunk
+  __shared__ int s_total_full;
   for (int i = threadIdx.x; i < E * W; i += blockDim.x) {
     const uint32_t wv = __ldcg(a.bitmap + i);
     words[i] = wv;
@@ -140,24 +144,28 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
     // so the result equals the sequential scan)
     const int per = (E + 31) / 32;
     const int base_chunks = a.n_shared ? (T + a.n_tile - 1) / a.n_tile : 0;
-    int c_cnt = 0, c_chk = 0, c_act = 0;
+    const int base_full = a.n_shared ? T / a.n_tile : 0;
+    int c_cnt = 0, c_chk = 0, c_act = 0, c_full = 0;
     for (int q = 0; q < per; ++q) {
       const int e = lane * per + q;
       if (e < E) {
         c_cnt += count[e];
         c_chk += (count[e] + a.n_tile - 1) / a.n_tile;
         c_act += count[e] > 0;
+        c_full += count[e] / a.n_tile;
       }
     }
-    int s_cnt = c_cnt, s_chk = c_chk;
+    int s_cnt = c_cnt, s_chk = c_chk, s_full = c_full;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int vc = __shfl_up_sync(0xffffffffu, s_cnt, o);
       const int vk = __shfl_up_sync(0xffffffffu, s_chk, o);
-      if (lane >= o) { s_cnt += vc; s_chk += vk; }
+      const int vf = __shfl_up_sync(0xffffffffu, s_full, o);
+      if (lane >= o) { s_cnt += vc; s_chk += vk; s_full += vf; }
     }
     int run = s_cnt - c_cnt;
     int crun = base_chunks + s_chk - c_chk;
+    int frun = base_full + s_full - c_full;
     for (int q = 0; q < per; ++q) {
       const int e = lane * per + q;
       if (e < E) {
@@ -165,14 +173,23 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
         if (a.offsets_r) a.offsets_r[e] = run;
         if (a.offsets_g) a.offsets_g[e + 1] = T + run;
         run += count[e];
+        cpre[e + 1] = crun;
+        fbase[e + 1] = frun;
         crun += (count[e] + a.n_tile - 1) / a.n_tile;
+        frun += count[e] / a.n_tile;
         if (a.chunk_prefix) a.chunk_prefix[e + 2] = crun;
       }
+    }
+    if (lane == 31) {
+      cpre[E + 1] = crun;
+      s_total_full = frun;
     }
     const int total = __shfl_sync(0xffffffffu, s_cnt, 31);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) c_act += __shfl_xor_sync(0xffffffffu, c_act, o);
     if (lane == 0) {
+      cpre[0] = 0;
+      fbase[0] = 0;
       if (a.offsets_g) a.offsets_g[0] = 0;
       if (a.chunk_prefix) { a.chunk_prefix[0] = 0; a.chunk_prefix[1] = base_chunks; }
       off[E] = total;
@@ -183,6 +200,28 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
     }
   }
   __syncthreads();
+  if (a.chunk_order) {
+    // The grouped GEMMs deal their tiles longest chunk first: the full chunks in
+    // chunk order, then each group's partial chunk by decreasing rows (ties
+    // toward the lower chunk).  Group 0 is the shared expert (T rows), group
+    // e + 1 expert e.
+    const int G = E + 1;
+    for (int g = threadIdx.x; g < G; g += blockDim.x) {
+      const int cnt = g == 0 ? (a.n_shared ? T : 0) : count[g - 1];
+      prow[g] = cnt % a.n_tile;
+      const int nfull = cnt / a.n_tile;
+      for (int j = 0; j < nfull; ++j) a.chunk_order[fbase[g] + j] = cpre[g] + j;
+    }
+    __syncthreads();
+    const int total_full = s_total_full;
+    for (int g = threadIdx.x; g < G; g += blockDim.x) {
+      const int r = prow[g];
+      if (r == 0) continue;
+      int rank = 0;
+      for (int g2 = 0; g2 < G; ++g2) rank += prow[g2] > r || (prow[g2] == r && g2 < g);
+      a.chunk_order[total_full + rank] = cpre[g + 1] - 1;
+    }
+  }
   for (int i0 = 0; i0 < T * k; i0 += 8 * kRouterThreads) {  // 8 index loads in flight per thread
     int ev[8];
 #pragma unroll
@@ -207,6 +246,8 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
   // the expert GEMMs' per-chunk ready counters start this layer at zero
   if (a.chunk_ready)
     for (int i = threadIdx.x; i < a.n_chunk_ready; i += blockDim.x) a.chunk_ready[i] = 0;
+  // and so do their tile counters
+  if (a.tile_counters && threadIdx.x < a.n_tile_counters) a.tile_counters[threadIdx.x] = 0;
   if (threadIdx.x == 0) *a.counter = 0;
 }
 
@@ -214,7 +255,7 @@ int router_max_smem_bytes() { return kRouterMaxSmem; }
 
 size_t router_smem_bytes(int T, int E) {
   const int W = (T + 31) / 32;
-  return (size_t)(2 * E * W + E + E + 1) * sizeof(int);
+  return (size_t)(2 * E * W + E + E + 1 + 3 * E + 4) * sizeof(int);
 }
 
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t s) {

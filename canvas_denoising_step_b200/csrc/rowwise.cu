@@ -499,7 +499,7 @@ constexpr int kMergeWarps = 32;
 
 __global__ void __launch_bounds__(kMergeWarps * 32) head_merge_kernel(
     const float* hm, const float* hs, const int* ha, int n_vblocks, int T, float* conf,
-    int32_t* tok) {
+    int32_t* tok, float* max_logit) {
   __shared__ float s_m[kMergeWarps][32], s_s[kMergeWarps][32];
   __shared__ int s_a[kMergeWarps][32];
   griddep_wait();
@@ -540,13 +540,15 @@ __global__ void __launch_bounds__(kMergeWarps * 32) head_merge_kernel(
     for (int w = 0; w < kMergeWarps; ++w) merge_stats(mt, st, at, s_m[w][lane], s_s[w][lane], s_a[w][lane]);
     conf[t] = 1.0f / st;
     tok[t] = at;
+    max_logit[t] = mt;
   }
 }
 
 cudaError_t launch_head_merge(const float* hm, const float* hs, const int* ha, int n_vblocks,
-                              int T, float* conf, int32_t* tok, cudaStream_t s) {
+                              int T, float* conf, int32_t* tok, float* max_logit,
+                              cudaStream_t s) {
   return launch_k(head_merge_kernel, dim3((T + 31) / 32), dim3(kMergeWarps * 32), 0, s, hm, hs,
-                  ha, n_vblocks, T, conf, tok);
+                  ha, n_vblocks, T, conf, tok, max_logit);
 }
 
 // ---------------------------------------------------------------- commit

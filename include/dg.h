@@ -186,6 +186,58 @@ int dg_canvas_step_host(dg_ctx* ctx, int32_t* canvas_host, int batch, int steps_
  * place.  Ends with a synchronisation and reports device errors. */
 int dg_denoise_block(dg_ctx* ctx, int32_t* canvas, int batch, int n_steps);
 
+/* Pages: "DiffusionGemma: The Diffusion Era Begins with 4x Faster Text
+ * Generation", Recommended Inference Settings (an entropy-bound sampler, at most
+ * 48 passes, temperature falling linearly from 0.8 to 0.4, entropy bound 0.1, a
+ * stop once the mean canvas entropy is below 0.005 with the high-probability
+ * tokens stable) and "DiffusionGemma: Exploring the Paradigm Shift in
+ * Non-Autoregressive Language Modeling", Serving in Production (the 0.005 halt
+ * once two consecutive passes agree).
+ * One entropy-bounded pass, pass `step` (0-based) of at most n_max, over `batch`
+ * canvases (dev int32 [batch][canvas_len], in place).  Its temperature is
+ * temp = 0.8 + (0.4 - 0.8) * step / (n_max - 1) (0.8 when n_max == 1).  Per row,
+ * the head gives the entropy H (nats) of softmax(logits / temp) over the
+ * vocabulary without the mask id, and the argmax token.  Per canvas:
+ *  - it stops when the mean of H over all its slots (summed in slot order in
+ *    double precision) is below 0.005 and every argmax equals the previous
+ *    pass's (pass 0 never stops);
+ *  - at a stop, or at the last pass (step == n_max - 1), every masked slot
+ *    takes its argmax token;
+ *  - otherwise the masked slots in order of (H, slot) are committed while
+ *    their running double-precision sum of H stays <= 0.1 (at least one), each
+ *    with a token drawn by inverse CDF: the first vocab index whose cumulative
+ *    probability (in vocab order) exceeds the slot's uniform.
+ * u: dev or host fp32 [batch][canvas_len] uniforms in [0, 1), one per slot.
+ * Pass 0 starts a block: it forgets the previous argmax and the canvases that
+ * ended.  A canvas that has stopped, filled up or passed its last pass is left
+ * unchanged by later passes of the block.  entropy_out (dev fp32
+ * [batch][canvas_len]), committed_out (dev uint8 [batch][canvas_len]) and
+ * stopped_out (dev uint8 [batch]) may be NULL.  Asynchronous like
+ * dg_canvas_step (graph recorded on the second call for a batch size). */
+int dg_eb_step(dg_ctx* ctx, int32_t* canvas, int batch, int step, int n_max, const float* u,
+               float* entropy_out, uint8_t* committed_out, uint8_t* stopped_out);
+
+/* Pages: as dg_eb_step.
+ * Entropy-bounded denoising of one block: dg_eb_step for step = 0, 1, ... until
+ * every canvas has stopped or filled up, or n_max passes ran.  u: dev fp32
+ * [n_max][batch][canvas_len] (pass s reads u + s * batch * canvas_len).
+ * passes_out (host int [batch], may be NULL) receives the passes each canvas
+ * took part in.  Reads the per-canvas state after every pass (one
+ * synchronisation per pass) and reports device errors at the end. */
+int dg_eb_denoise_block(dg_ctx* ctx, int32_t* canvas, int batch, int n_max, const float* u,
+                        int* passes_out);
+
+/* Pages: as dg_eb_step (the decisions of a pass).
+ * Test hook: the stop test and the commit of dg_eb_step on given per-slot
+ * entropies, argmax tokens and drawn tokens (all dev [batch][canvas_len]:
+ * fp32, int32, int32), with prev_argmax (dev int32, or NULL: no previous pass)
+ * and `last` (nonzero: the last allowed pass).  canvas in place;
+ * committed_out (dev uint8 [batch][canvas_len]) and stopped_out (dev uint8
+ * [batch]) may be NULL. */
+int dg_eb_commit(dg_ctx* ctx, const float* entropy, const int32_t* argmax, const int32_t* drawn,
+                 const int32_t* prev_argmax, int32_t* canvas, int batch, int last,
+                 uint8_t* committed_out, uint8_t* stopped_out);
+
 /* Pages: "Hands-On with Diffusion Gemma", Detailed Specs (input, post-attention
  * and pre-feedforward norms, attention, MoE) and "DiffusionGemma: The Diffusion
  * Era Begins ...", DiffusionGemma's Technical Architecture (bidirectional
@@ -277,6 +329,10 @@ int dg_commit(dg_ctx* ctx, const float* conf, int32_t* canvas, int batch, int st
  *   "h"        fp32 [T][d]        residual stream after the last layer run
  *   "tok"      int32 [T]          argmax token per row (after a pass)
  *   "conf"     fp32 [T]           confidence per row (after a pass)
+ *   "head_max" fp32 [T]           largest logit per row, mask id excluded (after a pass)
+ *   "entropy"  fp32 [T]           entropy per row (after an entropy-bounded pass)
+ *   "eb_drawn" int32 [T]          drawn token of each slot committed by the bound
+ *                                 (after an entropy-bounded pass; other rows stale)
  * and the weights (bf16, physical layouts):
  *   "embed"    [vocab][d]
  *   "wqkv:L"   [(Hq+2Hkv)*dh][d]  rows: q heads, then k heads, then v heads
