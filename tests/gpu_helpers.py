@@ -78,3 +78,25 @@ def bf16_bits(x: np.ndarray) -> np.ndarray:
 def oracle_weight_bits(cfg: dict, tid: int, shape, start=0) -> np.ndarray:
     return bf16_bits(orng.weight_tensor(cfg["seed"], tid, shape, cfg["weight_std"], True,
                                         start=start))
+
+
+ROUTER_TIE_TOL = 2e-2   # logit units; the device's logits differ from the oracle's by ~1e-3
+
+
+def router_flips(o_logits, o_idx, d_idx, tol=ROUTER_TIE_TOL) -> np.ndarray:
+    """Rows whose device top-k set differs from the oracle's own.  Each such row must
+    be a near-tie in the oracle's logits: every expert chosen by one side only lies
+    within `tol` of the oracle's k-th largest logit (the selection boundary).
+    Returns the boolean mask of flipped rows."""
+    o_logits = np.asarray(o_logits, dtype=np.float64)
+    k = o_idx.shape[1]
+    flipped = np.zeros(o_idx.shape[0], dtype=bool)
+    for t in range(o_idx.shape[0]):
+        a, b = set(int(e) for e in o_idx[t]), set(int(e) for e in d_idx[t])
+        if a == b:
+            continue
+        flipped[t] = True
+        boundary = np.sort(o_logits[t])[::-1][k - 1]
+        for e in a ^ b:
+            assert abs(o_logits[t, e] - boundary) < tol, (t, e, o_logits[t, e], boundary)
+    return flipped

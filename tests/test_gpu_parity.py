@@ -14,7 +14,7 @@ import torch
 import synth
 from oracle import model as om
 from oracle import rng as orng
-from tests.gpu_helpers import Ctx, bf16_bits, oracle_weight_bits, rel_l2
+from tests.gpu_helpers import Ctx, bf16_bits, oracle_weight_bits, rel_l2, router_flips
 
 pytestmark = pytest.mark.gpu
 
@@ -188,20 +188,19 @@ def _layer_check(name, layer, **kw):
         # MoE on the device's x2 and selection
         y, _, _, _ = om.moe_ffn(oc, W, x2.astype(np.float64), forced_idx=idx)
         report["moe_out"] = rel_l2(got.reshape(T, d), h1 + y)
-        # whole layer, oracle end to end
-        flips = int((tr["idx"] != idx).any(axis=1).sum())
-        report["layer"] = rel_l2(got, ref)
-        report["router_rows_flipped"] = flips
+        # whole layer, oracle end to end; a row whose top-k set differs must be a
+        # near-tie in the oracle's own logits, and every other row matches
+        flipped = router_flips(tr["router_logits"], tr["idx"], idx)
+        keep = ~flipped.reshape(B, Tc)
+        report["layer"] = rel_l2(got[keep], ref[keep])
+        report["router_rows_flipped"] = int(flipped.sum())
         print(name, layer, report)
         for key in ("q", "k", "v", "attn"):
             assert max(report[key]) < LAYER_TOL, (key, report)
         for key in ("x2", "moe_out"):
             assert report[key] < LAYER_TOL, (key, report)
         assert report["logits"] < 1e-4, report
-        if flips == 0:
-            assert report["layer"] < LAYER_TOL, report
-        else:
-            assert report["layer"] < 5 * LAYER_TOL, report
+        assert report["layer"] < LAYER_TOL, report
         return report
     finally:
         c.close()
@@ -218,6 +217,51 @@ def test_layer_parity_rope_off_and_no_shared():
 
 # ----------------------------------------------------------------------------- full step
 
+LOGIT_TOL = 5e-2     # max-abs on logits
+
+
+def _oracle_pass_logits(oc, canvas0, kvs):
+    """The oracle's own pass up to the full logits: embedding, every block, the final
+    norm, then hn E^T over the whole vocabulary (small vocabularies only)."""
+    B, Tc = canvas0.shape
+    h = om.embedding_rows(oc, canvas0.reshape(-1)).reshape(B, Tc, oc.d_model)
+    for l in range(oc.n_layers):
+        h = om.layer_forward(oc, om.layer_weights(oc, l), h, kvs[l][0], kvs[l][1])
+    hn = om.rmsnorm(h, np.ones(oc.d_model), oc.rms_eps).reshape(B * Tc, oc.d_model)
+    return hn @ om.embedding_block(oc, 0, oc.vocab).T
+
+
+def _assert_commit_matches_up_to_near_ties(dev_canvas, canvas0, o_logits, mask_id, S, tol):
+    """The device's committed slots and tokens equal the oracle's own commit, except
+    where the oracle itself is within `tol` of a tie: a slot whose confidence (log)
+    is within tol of the commit boundary may be on either side, and a token whose
+    top-two logits are within tol may be either of the two."""
+    lg = np.array(o_logits, dtype=np.float64, copy=True)
+    lg[:, mask_id] = -np.inf
+    B, Tc = canvas0.shape
+    top2 = np.sort(lg, axis=1)[:, -2:]
+    o_conf, o_tok, _, _ = om.logit_stats(o_logits, mask_id)
+    o_can, _ = om.commit(canvas0, o_conf.reshape(B, Tc), o_tok.reshape(B, Tc), S, mask_id)
+    lc = np.log(o_conf).reshape(B, Tc)
+    gap = (top2[:, 1] - top2[:, 0]).reshape(B, Tc)
+    n_near = 0
+    for b in range(B):
+        masked = np.nonzero(canvas0[b] == mask_id)[0]
+        k = om.commit_count(len(masked), S)
+        boundary = np.sort(lc[b, masked])[::-1][k - 1]
+        dev_set = set(np.nonzero(dev_canvas[b] != canvas0[b])[0])
+        o_set = set(np.nonzero(o_can[b] != canvas0[b])[0])
+        assert len(dev_set) == k
+        for i in dev_set ^ o_set:
+            assert abs(lc[b, i] - boundary) < tol, (b, i, lc[b, i], boundary)
+            n_near += 1
+        for i in dev_set & o_set:
+            if dev_canvas[b, i] != o_can[b, i]:
+                assert gap[b, i] < tol, (b, i, gap[b, i])
+                n_near += 1
+    return n_near
+
+
 @pytest.mark.parametrize("name", ["tiny", "ragged"])
 def test_canvas_step_head_and_commit(name):
     cfg = gpu_cfg(name)
@@ -233,23 +277,33 @@ def test_canvas_step_head_and_commit(name):
         c.dg.dg_sync(c.ctx)
         hn = c.fetch("hn", torch.bfloat16, (T, cfg["d_model"]))
         tok = c.fetch("tok", torch.int32, (T,))
+        mx = c.fetch("head_max", torch.float32, (T,))
         conf_np = conf.cpu().numpy()
         # vocab head on the device's final hidden states
         rconf, rtok, rm, _ = om.head_reduce(oc, hn.astype(np.float64))
         assert np.allclose(conf_np.ravel(), rconf, rtol=1e-3)
         assert np.array_equal(tok, rtok)
+        assert np.abs(mx - rm).max() < 1e-3
         # commit on the device's confidences: bit-exact
         ref_can, ref_com = om.commit(canvas0, conf_np, tok.reshape(B, Tc), S, cfg["mask_id"])
         assert np.array_equal(canvas.cpu().numpy(), ref_can)
         assert np.array_equal(com.cpu().numpy().astype(bool), ref_com)
-        # whole pass against the oracle end to end
+        # whole pass against the oracle end to end: logits, confidences, the commit
         kvs = [c.kv_np(l) for l in range(cfg["n_layers"])]
-        o_can, o_conf, o_tok, _ = om.canvas_step(oc, canvas0, [kv[0] for kv in kvs],
-                                                 [kv[1] for kv in kvs], S)
-        err = np.abs(np.log(conf_np) - np.log(o_conf)).max()
-        print(name, "end-to-end max |log conf diff|", err,
-              "argmax agreement", float((o_tok == tok.reshape(B, Tc)).mean()))
-        assert err < 5e-2
+        o_logits = _oracle_pass_logits(oc, canvas0, kvs)
+        o_conf, o_tok, o_m, _ = om.logit_stats(o_logits, cfg["mask_id"])
+        err_m = np.abs(mx - o_m).max()
+        err = np.abs(np.log(conf_np.ravel()) - np.log(o_conf)).max()
+        n_near = _assert_commit_matches_up_to_near_ties(canvas.cpu().numpy(), canvas0, o_logits,
+                                                        cfg["mask_id"], S, LOGIT_TOL)
+        print(name, "end-to-end max |max-logit diff|", err_m, "max |log conf diff|", err,
+              "argmax agreement", float((o_tok == tok).mean()), "near-tie exemptions", n_near)
+        assert err_m < LOGIT_TOL
+        assert err < LOGIT_TOL
+        # the oracle's own full pass gives the same canvas up to those near-ties
+        o_can, _, _, _ = om.canvas_step(oc, canvas0, [kv[0] for kv in kvs],
+                                        [kv[1] for kv in kvs], S)
+        assert (o_can != canvas.cpu().numpy()).sum() <= n_near
     finally:
         c.close()
 
