@@ -40,16 +40,17 @@ WORKLOAD = "stack"
 
 
 def workload_desc(cfg):
+    skew = f", Zipf({cfg['zipf_s']}) expert popularity" if cfg.get("zipf_s") else ""
     return (f"{cfg['n_layers']}-layer canvas denoising stack: d_model {cfg['d_model']}, "
             f"{cfg['n_q_heads']}q/{cfg['n_kv_heads']}kv heads x {cfg['head_dim']}, "
             f"{cfg['n_experts']} experts top-{cfg['top_k']} + {cfg['n_shared']} shared "
             f"(width {cfg['d_ff']}), vocab {cfg['vocab']} tied, canvas {cfg['canvas_len']}, "
             f"prompt K/V {cfg['prompt_len']} per layer (window {cfg['window']} on 5 of 6 layers), "
-            f"batch {cfg['batch']}, {cfg['steps']} steps per block")
+            f"batch {cfg['batch']}, {cfg['steps']} steps per block{skew}")
 
 
 def config_json(cfg, n_gpus):
-    return {"workload": workload_desc(cfg), "name": WORKLOAD, "batch": cfg["batch"],
+    return {"workload": workload_desc(cfg), "name": cfg["name"], "batch": cfg["batch"],
             "canvas_len": cfg["canvas_len"], "prompt_len": cfg["prompt_len"],
             "steps_per_block": cfg["steps"], "n_layers": cfg["n_layers"],
             "l2": "inputs larger than L2: ~50 GB of weights streamed from HBM every step",
@@ -86,6 +87,34 @@ def gateup_bytes_per_launch(cfg, active_experts=None):
     return (act + cfg["n_shared"]) * 2 * F * d * 2 + rows * d * 2 + rows * F * 2
 
 
+def gateup_flops_per_launch(cfg):
+    """2 * rows * 2F * d over the shared expert's T rows and the k * T routed rows."""
+    d, F, k = cfg["d_model"], cfg["d_ff"], cfg["top_k"]
+    T = cfg["batch"] * cfg["canvas_len"]
+    return 2 * (k + cfg["n_shared"]) * T * 2 * F * d
+
+
+def gateup_roofline(cfg, avg_launch_ms, active_experts, peaks):
+    """The gate/up GEMM against its own roofline: bytes over the measured copy
+    bandwidth, or FLOPs over the measured sustained bf16 throughput, whichever
+    takes longer for its algorithmic work."""
+    nbytes = gateup_bytes_per_launch(cfg, active_experts)
+    flops = gateup_flops_per_launch(cfg)
+    t = avg_launch_ms / 1e3
+    hbm, tflops, kind = peaks
+    if flops / (tflops * 1e12) > nbytes / (hbm * 1e9):
+        achieved = flops / t / 1e12
+        return {"bound": "tensor", "kernel": "gemm_gateup", "achieved": achieved,
+                "peak": tflops, "unit": "TFLOP/s", "frac": achieved / tflops,
+                "peak_source": kind + " (sustained bf16)", "traffic": None,
+                "algorithmic_flops_per_launch": flops, "avg_launch_ms": avg_launch_ms}
+    achieved = nbytes / t / 1e9
+    return {"bound": "hbm", "kernel": "gemm_gateup", "achieved": achieved, "peak": hbm,
+            "unit": "GB/s", "frac": achieved / hbm, "peak_source": kind,
+            "traffic": load_traffic("gemm_gateup") if cfg["name"] == "stack" else None,
+            "algorithmic_bytes_per_launch": nbytes, "avg_launch_ms": avg_launch_ms}
+
+
 def flops_per_step(cfg):
     d, F, E, k = cfg["d_model"], cfg["d_ff"], cfg["n_experts"], cfg["top_k"]
     dh, Hq, Hkv = cfg["head_dim"], cfg["n_q_heads"], cfg["n_kv_heads"]
@@ -103,11 +132,13 @@ def flops_per_step(cfg):
 # ----------------------------------------------------------------------------- peaks, clocks, traffic
 
 def load_peaks():
+    """(HBM GB/s, sustained bf16 TFLOP/s, "measured" | "fallback")."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         j = json.load(open(p))
-        return float(j["hbm_gbs"]), "measured"
-    return 6650.0, "fallback"
+        return (float(j["hbm_gbs"]), float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                "measured")
+    return 6650.0, 1400.0, "fallback"
 
 
 def kernel_src_sha():
@@ -226,22 +257,27 @@ def oracle_sample(cfg, layers, vocab_fraction_den, seed_rows=0):
     from oracle import model as om
     oc = om.OracleConfig.from_dict(cfg)
     B, Tc, d = cfg["batch"], cfg["canvas_len"], cfg["d_model"]
-    h = synth.hidden_states(cfg).float().numpy().astype(np.float64).reshape(B, Tc, d)
+    # with several canvases, one of them is run and the time scaled by the batch
+    h = synth.hidden_states(cfg).float().numpy().astype(np.float64).reshape(B, Tc, d)[:1]
+    bias = None
+    if cfg.get("zipf_s"):
+        bias = synth.zipf_router_bias(cfg["n_experts"], cfg["zipf_s"]).numpy()
     times = []
     for l in layers:
         Wc = _CachedWeights(oc, l)
         k, v = synth.prompt_kv(cfg, l)
-        kp, vp = k.float().numpy().astype(np.float64), v.float().numpy().astype(np.float64)
+        kp = k[:1].float().numpy().astype(np.float64)
+        vp = v[:1].float().numpy().astype(np.float64)
         t0 = time.perf_counter()
-        om.layer_forward(oc, Wc.W, h, kp, vp)
-        times.append(time.perf_counter() - t0)
+        om.layer_forward(oc, Wc.W, h, kp, vp, router_bias=bias)
+        times.append((time.perf_counter() - t0) * B)
     nv = cfg["vocab"] // vocab_fraction_den
     Eb = om.embedding_block(oc, 0, nv)
-    hn = om.rmsnorm(h.reshape(B * Tc, d), 1.0, oc.rms_eps)
+    hn = om.rmsnorm(h.reshape(Tc, d), 1.0, oc.rms_eps)
     t0 = time.perf_counter()
     lg = hn @ Eb.T
     om.logit_stats(lg, oc.mask_id)
-    t_head = time.perf_counter() - t0
+    t_head = (time.perf_counter() - t0) * B
     return times, t_head
 
 
@@ -264,8 +300,9 @@ def cpu_baseline(cfg):
     t_step = (L - n_glob) * t_loc + n_glob * t_glob + 32 * t_head
     value = cfg["batch"] * cfg["canvas_len"] / (cfg["steps"] * t_step)
     return {"value": value, "unit": "canvas tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": (f"one local and one global full-size layer (256 canvas rows) and 1/32 of "
-                       f"the vocab head, weights pre-drawn; pass time extrapolated as "
+            "sample": (f"one local and one global full-size layer (256 canvas rows; times "
+                       f"{cfg['batch']} for the batch) and 1/32 of the vocab head, weights "
+                       f"pre-drawn; pass time extrapolated as "
                        f"{L - n_glob} local + {n_glob} global layers + 32 head slices "
                        f"= {t_step:.1f} s")}
 
@@ -299,6 +336,21 @@ def run_reference(args, cfg, rank, world):
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def step_roofline(cfg, step_ms, active_avg, peaks):
+    """A whole pass against max(bytes / HBM bandwidth, FLOPs / sustained bf16)."""
+    hbm, tflops, _ = peaks
+    nbytes = bytes_per_step(cfg, active_avg)
+    flops = flops_per_step(cfg)
+    t_hbm = nbytes / (hbm * 1e9) * 1e3
+    t_tc = flops / (tflops * 1e12) * 1e3
+    return {"bytes": nbytes, "flops": flops, "active_experts_per_layer": active_avg,
+            "bytes_if_all_experts": bytes_per_step(cfg),
+            "achieved_gbs": nbytes / (step_ms / 1e3) / 1e9,
+            "frac_of_hbm": nbytes / (step_ms / 1e3) / 1e9 / hbm,
+            "bound": "hbm" if t_hbm >= t_tc else "tensor",
+            "roofline_ms": max(t_hbm, t_tc), "frac_of_roofline": max(t_hbm, t_tc) / step_ms}
 
 
 def max_over_ranks(values, world, device):
@@ -338,6 +390,9 @@ def run_ours(args, cfg, rank, world, local_rank):
             dg.dg_set_prompt_kv(ctx, l, kd.data_ptr(), vd.data_ptr(), B, cfg["prompt_len"])
         canvas0 = synth.initial_canvas(cfg).to(dev)
         canvas = canvas0.clone()
+        if cfg.get("zipf_s"):
+            bias = synth.zipf_router_bias(cfg["n_experts"], cfg["zipf_s"]).to(dev)
+            dg.dg_set_router_bias(ctx, bias.data_ptr())
     stream.synchronize()
 
     def run_steps(n, start=0):
@@ -412,10 +467,9 @@ def run_ours(args, cfg, rank, world, local_rank):
         return
 
     value = canvas_throughput(world, B, Tc, args.steps, S, t_max)
-    peak, peak_kind = load_peaks()
+    peaks = load_peaks()
+    peak = peaks[0]
     gu_ms, gu_n = kern.get("gemm_gateup", (float("nan"), 1))
-    gu_bytes = gateup_bytes_per_launch(cfg, active_avg)
-    achieved = gu_bytes / (gu_ms / gu_n / 1e3) / 1e9
     step_bytes = bytes_per_step(cfg, active_avg)
     step_ms = t_max / args.steps
     total_prof = sum(v[0] for v in kern.values())
@@ -425,17 +479,8 @@ def run_ours(args, cfg, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": config_json(cfg, world),
-        "roofline": {"bound": "hbm", "kernel": "gemm_gateup", "achieved": achieved,
-                     "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_source": peak_kind, "traffic": load_traffic("gemm_gateup"),
-                     "algorithmic_bytes_per_launch": gu_bytes,
-                     "avg_launch_ms": gu_ms / gu_n},
-        "step_roofline": {"bytes": step_bytes, "flops": flops_per_step(cfg),
-                          "active_experts_per_layer": active_avg,
-                          "bytes_if_all_experts": bytes_per_step(cfg),
-                          "achieved_gbs": step_bytes / (step_ms / 1e3) / 1e9,
-                          "frac_of_hbm": step_bytes / (step_ms / 1e3) / 1e9 / peak,
-                          "roofline_ms": step_bytes / (peak * 1e9) * 1e3},
+        "roofline": gateup_roofline(cfg, gu_ms / gu_n, active_avg, peaks),
+        "step_roofline": step_roofline(cfg, step_ms, active_avg, peaks),
         "kernels_ms_per_step": {k: v[0] / args.steps for k, v in
                                 sorted(kern.items(), key=lambda kv: -kv[1][0])},
         "profiled_ms_per_step": total_prof / args.steps,
@@ -450,10 +495,33 @@ def run_ours(args, cfg, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def layer_bytes(cfg, layer, active_experts):
+    """Algorithmic HBM bytes of one block: its dense weights, the shared expert and the
+    routed experts that receive rows, and the visible prompt K/V."""
+    d, F, E = cfg["d_model"], cfg["d_ff"], cfg["n_experts"]
+    dh, Hq, Hkv = cfg["head_dim"], cfg["n_q_heads"], cfg["n_kv_heads"]
+    P = cfg["prompt_len"]
+    vis = P if (layer + 1) % cfg["global_every"] == 0 else min(cfg["window"], P)
+    dense = 2 * ((Hq + 2 * Hkv) * dh * d + d * Hq * dh + E * d)
+    return dense + 2 * (active_experts + cfg["n_shared"]) * 3 * F * d + \
+        2 * cfg["batch"] * Hkv * vis * dh * 2
+
+
+def layer_flops(cfg, layer):
+    d, F, E, k = cfg["d_model"], cfg["d_ff"], cfg["n_experts"], cfg["top_k"]
+    dh, Hq, Hkv, Tc = cfg["head_dim"], cfg["n_q_heads"], cfg["n_kv_heads"], cfg["canvas_len"]
+    T = cfg["batch"] * Tc
+    P = cfg["prompt_len"]
+    vis = P if (layer + 1) % cfg["global_every"] == 0 else min(cfg["window"], P)
+    return (2 * T * d * ((Hq + 2 * Hkv) * dh + Hq * dh + E) +
+            4 * cfg["batch"] * Hq * Tc * (vis + Tc) * dh + 2 * T * (k + cfg["n_shared"]) * 3 * F * d)
+
+
 def run_layer_case(args, cfg):
     """One decoder block (dg_layer_forward) on N(0,1) hidden states -- the
-    single-layer workload -- timed with CUDA events, with the per-kernel table.
-    Not the headline line; used for kernel studies and focused ncu captures."""
+    single-layer workload -- timed with CUDA events over K calls after W warm-ups,
+    with the clocks of the timed region, the per-kernel table, the block's roofline
+    and the gate/up GEMM's, and the oracle timed on the same block."""
     import torch
     import canvas_denoising_step_b200 as dg
     import synth
@@ -473,13 +541,24 @@ def run_layer_case(args, cfg):
         for _ in range(args.warmup):
             dg.dg_layer_forward(ctx, layer, x.data_ptr(), out.data_ptr(), T)
         dg.dg_sync(ctx)
+        launches = dg.dg_last_launch_count(ctx)
+        clocks = ClockSampler(0)
+        clocks.start()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        stream.synchronize()
+        clocks.mark_begin()
         e0.record(stream)
         for _ in range(args.steps):
             dg.dg_layer_forward(ctx, layer, x.data_ptr(), out.data_ptr(), T)
         e1.record(stream)
         stream.synchronize()
+        clocks.mark_end()
+        clk = clocks.stop()
         ms = e0.elapsed_time(e1) / args.steps
+        dg.dg_sync(ctx)
+        act0 = torch.empty(cfg["n_layers"], dtype=torch.int32, device="cuda")
+        dg.dg_debug_tensor(ctx, "expert_active", act0.data_ptr(), 4 * cfg["n_layers"])
+        act_before = int(act0[layer].item())
         dg.dg_profile_enable(ctx, 1)
         for _ in range(args.steps):
             dg.dg_layer_forward(ctx, layer, x.data_ptr(), out.data_ptr(), T)
@@ -487,16 +566,129 @@ def run_layer_case(args, cfg):
         while (name := dg.dg_kernel_name(i)) is not None:
             tot, cnt = dg.dg_profile_read(ctx, name)
             if cnt:
-                kern[name] = tot / args.steps
+                kern[name] = (tot, cnt)
             i += 1
         dg.dg_profile_enable(ctx, 0)
         act = torch.empty(cfg["n_layers"], dtype=torch.int32, device="cuda")
         dg.dg_debug_tensor(ctx, "expert_active", act.data_ptr(), 4 * cfg["n_layers"])
+        active = int(act[layer].item()) / args.steps
         dg.dg_destroy(ctx)
-    print(json.dumps({"case": "layer_forward", "workload": args.workload, "layer": layer,
-                      "ms_per_layer": ms, "expert_active": int(act[layer].item()) // args.steps,
-                      "kernels_ms": dict(sorted(kern.items(), key=lambda kv: -kv[1]))}),
-          flush=True)
+    del act_before
+    peaks = load_peaks()
+    hbm, tflops, kind = peaks
+    nbytes, flops = layer_bytes(cfg, layer, active), layer_flops(cfg, layer)
+    t_roof = max(nbytes / (hbm * 1e9), flops / (tflops * 1e12)) * 1e3
+    gu_ms, gu_n = kern.get("gemm_gateup", (float("nan"), 1))
+    line = {
+        "metric": "decoder-block latency on 1 B200 (single-layer workload); % of its roofline",
+        "value": ms, "unit": "ms", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": (f"one {'global' if (layer + 1) % cfg['global_every'] == 0 else 'local'} "
+                                f"decoder block: d_model {cfg['d_model']}, {cfg['n_q_heads']}q/"
+                                f"{cfg['n_kv_heads']}kv x {cfg['head_dim']}, {cfg['n_experts']} "
+                                f"experts top-{cfg['top_k']} + {cfg['n_shared']} shared (width "
+                                f"{cfg['d_ff']}), canvas {Tc} x batch {B}, prompt K/V "
+                                f"{cfg['prompt_len']}, hidden states N(0,1), no vocab head"),
+                   "name": cfg["name"], "layer": layer,
+                   "l2": "inputs larger than L2: 1.6 GB of block weights per call",
+                   "parallelism": "single"},
+        "roofline": gateup_roofline(cfg, gu_ms / gu_n, active, peaks),
+        "step_roofline": {"bytes": nbytes, "flops": flops, "active_experts": active,
+                          "roofline_ms": t_roof, "frac_of_roofline": t_roof / ms,
+                          "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
+                          "bound": "hbm" if nbytes / hbm / 1e9 >= flops / tflops / 1e12
+                          else "tensor"},
+        "kernels_ms_per_step": {k2: v2[0] / args.steps for k2, v2 in
+                                sorted(kern.items(), key=lambda kv: -kv[1][0])},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline:
+        (t_layer,), _ = oracle_sample(cfg, [layer], cfg["vocab"])
+        line["cpu_baseline"] = {"value": t_layer * 1e3, "unit": "ms", "cores": blas_threads(),
+                                "kind": "oracle",
+                                "sample": "the same block on the same hidden states, in full "
+                                          "(weights pre-drawn; the head term is one vocab row)"}
+    print(json.dumps(line), flush=True)
+
+
+def run_eb_case(args, cfg):
+    """Entropy-bounded passes (dg_eb_step) on the workload: K passes after W warm-ups,
+    each pass the whole stack, the head at the pass's temperature with the entropy
+    reduction, the stop test and the bounded commit with its draw.  Reports the pass
+    latency against the pass's roofline (the same bytes and FLOPs as a fixed-step
+    pass: the entropy terms add no HBM traffic)."""
+    import numpy as np
+    import torch
+    import canvas_denoising_step_b200 as dg
+    import synth
+
+    torch.cuda.set_device(0)
+    stream = torch.cuda.Stream()
+    B, Tc, L = cfg["batch"], cfg["canvas_len"], cfg["n_layers"]
+    n_max = 48
+    with torch.cuda.stream(stream):
+        ctx = dg.dg_create(dg.config_from_dict(cfg), stream.cuda_stream)
+        dg.dg_init_weights(ctx, cfg["seed"])
+        kv = []
+        for l in range(L):
+            k, v = synth.prompt_kv(cfg, l)
+            kd, vd = k.cuda(), v.cuda()
+            kv.append((kd, vd))
+            dg.dg_set_prompt_kv(ctx, l, kd.data_ptr(), vd.data_ptr(), B, cfg["prompt_len"])
+        g = np.random.default_rng(7)
+        u = torch.from_numpy(g.uniform(size=(n_max, B, Tc)).astype(np.float32)).cuda()
+        canvas0 = synth.initial_canvas(cfg).cuda()
+        canvas = canvas0.clone()
+
+        def passes(n):
+            for s in range(n):
+                step = s % n_max
+                if step == 0:
+                    canvas.copy_(canvas0, non_blocking=True)
+                dg.dg_eb_step(ctx, canvas.data_ptr(), B, step, n_max,
+                              u[step].data_ptr())
+
+        passes(args.warmup)
+        dg.dg_sync(ctx)
+        launches = dg.dg_last_launch_count(ctx)
+        clocks = ClockSampler(0)
+        clocks.start()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        stream.synchronize()
+        clocks.mark_begin()
+        e0.record(stream)
+        passes(args.steps)
+        e1.record(stream)
+        stream.synchronize()
+        clocks.mark_end()
+        clk = clocks.stop()
+        ms = e0.elapsed_time(e1) / args.steps
+        dg.dg_sync(ctx)
+        dg.dg_profile_enable(ctx, 1)
+        passes(args.steps)
+        kern, i = {}, 0
+        while (name := dg.dg_kernel_name(i)) is not None:
+            tot, cnt = dg.dg_profile_read(ctx, name)
+            if cnt:
+                kern[name] = tot / args.steps
+            i += 1
+        dg.dg_profile_enable(ctx, 0)
+        act = torch.empty(L, dtype=torch.int32, device="cuda")
+        dg.dg_debug_tensor(ctx, "expert_active", act.data_ptr(), 4 * L)
+        active = float(act.sum().item()) / (args.steps * L)
+        dg.dg_destroy(ctx)
+    peaks = load_peaks()
+    print(json.dumps({
+        "metric": "entropy-bounded pass latency on 1 B200; % of the pass roofline",
+        "value": ms, "unit": "ms", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": dict(config_json(cfg, 1), sampler="entropy-bounded, 48 passes at most"),
+        "step_roofline": step_roofline(cfg, ms, active, peaks),
+        "kernels_ms_per_step": dict(sorted(kern.items(), key=lambda kv: -kv[1])),
+        "gpu_launches": launches * args.steps, "clocks": clk}), flush=True)
 
 
 def main():
@@ -510,6 +702,9 @@ def main():
     ap.add_argument("--case", choices=["step", "layer"], default="step",
                     help="step: full canvas passes (the headline); layer: dg_layer_forward")
     ap.add_argument("--layer", type=int, default=0)
+    ap.add_argument("--sampler", choices=["fixed", "eb"], default="fixed",
+                    help="fixed: k = ceil(r / steps_left) commits (the headline); eb: "
+                         "entropy-bounded passes")
     ap.add_argument("--set", action="append", default=[], metavar="KEY=INT",
                     help="override an integer workload field (kernel studies only)")
     args = ap.parse_args()
@@ -520,6 +715,9 @@ def main():
                                          for kv in args.set})
     if args.case == "layer":
         run_layer_case(args, cfg)
+        return
+    if args.sampler == "eb":
+        run_eb_case(args, cfg)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
