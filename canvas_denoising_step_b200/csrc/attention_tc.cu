@@ -43,8 +43,8 @@ struct AttnSmem {
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQ;                  // [stage] K
   static constexpr int kVOff = kKOff + kStages * kKV;
-  static constexpr int kPOff = kVOff + kStages * kKV;
-  static constexpr int kBarOff = kPOff + kP;
+  static constexpr int kPOff = kVOff + kStages * kKV;   // [2] P tiles
+  static constexpr int kBarOff = kPOff + 2 * kP;
   static constexpr int kBytes = kBarOff + 256;
 };
 
@@ -64,14 +64,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
   const uint32_t bars = sbase + L::kBarOff;
   // barrier slots (8 bytes each)
   const uint32_t q_full = bars + 0;
-  auto kv_full = [&](int s) { return bars + 8u * (1 + s); };
-  auto kv_empty = [&](int s) { return bars + 8u * (3 + s); };
+  // K and V of a block have rings of their own: K(j) is released as soon as
+  // QK^T(j) has read it, V(j) after PV(j), so each load is issued about two
+  // blocks before it is used
+  auto k_full = [&](int s) { return bars + 8u * (1 + s); };
+  auto k_empty = [&](int s) { return bars + 8u * (3 + s); };
+  auto v_full = [&](int s) { return bars + 8u * (13 + s); };
+  auto v_empty = [&](int s) { return bars + 8u * (15 + s); };
   auto s_full = [&](int s) { return bars + 8u * (5 + s); };
   auto s_free = [&](int s) { return bars + 8u * (7 + s); };
-  const uint32_t p_full = bars + 8u * 9;
-  const uint32_t pv_done = bars + 8u * 10;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOff + 8 * 12);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kBarOff + 8 * 12 + 4);
+  auto p_full = [&](int b) { return bars + 8u * (9 + b); };     // P tile b written
+  auto pv_done = [&](int b) { return bars + 8u * (11 + b); };   // the PV MMAs reading P tile b done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOff + 8 * 17);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kBarOff + 8 * 17 + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x, chunk = blockIdx.y;
@@ -84,23 +89,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
   const int jb0 = (int)(((long long)chunk * nb) / a.n_chunks);
   const int jb1 = (int)(((long long)(chunk + 1) * nb) / a.n_chunks);
   const int n_local = jb1 - jb0;
-  // TMEM: O at [0, DH); then two S buffers, each split into kSChains
-  // independent accumulator chains of kBN columns (the k16 steps of QK^T
-  // alternate between chains so consecutive MMAs do not depend on each other).
-  constexpr int kSChains = (DH + 2 * 4 * kBN <= 512) ? 4 : 2;
-  constexpr uint32_t kTmemCols = (DH + 2 * kSChains * kBN <= 256) ? 256 : 512;
+  // TMEM: O at [0, DH); then two S buffers (the next QK^T runs while the
+  // softmax reads the last one), each split into two independent accumulator
+  // chains of kBN columns: the k16 steps of QK^T alternate between them, so
+  // consecutive MMAs do not wait for one another.
+  constexpr int kSChains = 2;
+  constexpr int kSBufs = 2;
+  constexpr uint32_t kTmemCols = (DH + kSBufs * kSChains * kBN <= 256) ? 256 : 512;
   constexpr uint32_t kOCol = 0, kSCol = DH;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(kv_full(s), 1);
-      mbar_init(kv_empty(s), 1);
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
       mbar_init(s_full(s), 1);
       mbar_init(s_free(s), 4);
     }
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(p_full(b), 4);
+      mbar_init(pv_done(b), 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&mapQ);
@@ -120,12 +131,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
   // The prompt K/V is set before the pass and never written by it: the
   // producer issues the first ring stages of prompt blocks before the grid
   // wait (fresh barriers, no empty waits); q and the canvas K/V come after it.
-  auto issue_kv = [&](int j) {
-    const int st = j % kStages;
+  auto block_src = [&](int j, const CUtensorMap*& mk, const CUtensorMap*& mv, int& row) {
     const int jg = jb0 + j;
-    const CUtensorMap* mk;
-    const CUtensorMap* mv;
-    int row;
     if (jg < nbp) {
       mk = &mapKp; mv = &mapVp;
       row = (b * a.Hkv + g) * a.P + (a.P - a.n_vis) + jg * kBN;
@@ -133,15 +140,32 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
       mk = &mapKc; mv = &mapVc;
       row = (b * a.Hkv + g) * a.Tc + (jg - nbp) * kBN;
     }
-    mbar_arrive_expect_tx(kv_full(st), (uint32_t)(2 * L::kKV));
-    for (int c = 0; c < DH / 64; ++c) {
-      tma_load_2d(sbase + L::kKOff + st * L::kKV + c * (kBN * 128), mk, kv_full(st), c * 64, row);
-      tma_load_2d(sbase + L::kVOff + st * L::kKV + c * (kBN * 128), mv, kv_full(st), c * 64, row);
-    }
+  };
+  auto issue_k = [&](int j) {
+    const int st = j % kStages;
+    const CUtensorMap *mk, *mv;
+    int row;
+    block_src(j, mk, mv, row);
+    mbar_arrive_expect_tx(k_full(st), (uint32_t)L::kKV);
+    for (int c = 0; c < DH / 64; ++c)
+      tma_load_2d(sbase + L::kKOff + st * L::kKV + c * (kBN * 128), mk, k_full(st), c * 64, row);
+  };
+  auto issue_v = [&](int j) {
+    const int st = j % kStages;
+    const CUtensorMap *mk, *mv;
+    int row;
+    block_src(j, mk, mv, row);
+    mbar_arrive_expect_tx(v_full(st), (uint32_t)L::kKV);
+    for (int c = 0; c < DH / 64; ++c)
+      tma_load_2d(sbase + L::kVOff + st * L::kKV + c * (kBN * 128), mv, v_full(st), c * 64, row);
   };
   int pre_kv = 0;
   if (warp == 0 && lane == 0)
-    while (pre_kv < kStages && pre_kv < n_local && jb0 + pre_kv < nbp) issue_kv(pre_kv++);
+    while (pre_kv < kStages && pre_kv < n_local && jb0 + pre_kv < nbp) {
+      issue_k(pre_kv);
+      issue_v(pre_kv);
+      ++pre_kv;
+    }
   griddep_wait();
   griddep_launch();
 
@@ -153,18 +177,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
       for (int c = 0; c < DH / 64; ++c)
         tma_load_2d(sbase + L::kQOff + c * (kRows * 128), &mapQ, q_full, c * 64, q_row0);
       bool ok = true;
-      int issued = pre_kv;
-      for (int j = pre_kv; j < n_local && ok; ++j) {
-        const int st = j % kStages;
-        const uint32_t par = (uint32_t)((j / kStages) & 1) ^ 1u;
-        if (!mbar_wait(kv_empty(st), par, abort_flag, a.err)) { ok = false; break; }
-        issue_kv(j);
-        ++issued;
+      // K(j) waits for QK^T(j - 2), V(j) for PV(j - 2); V is issued one block
+      // behind K, which is the order in which the MMAs free their stages
+      int ik = pre_kv, iv = pre_kv;
+      while (ok && (ik < n_local || iv < n_local)) {
+        if (ik < n_local) {
+          if (!mbar_wait(k_empty(ik % kStages), (uint32_t)((ik / kStages) & 1) ^ 1u, abort_flag, a.err)) {
+            ok = false;
+            break;
+          }
+          issue_k(ik++);
+        }
+        if (iv < n_local && (iv < ik - 1 || ik == n_local)) {
+          if (!mbar_wait(v_empty(iv % kStages), (uint32_t)((iv / kStages) & 1) ^ 1u, abort_flag, a.err)) {
+            ok = false;
+            break;
+          }
+          issue_v(iv++);
+        }
       }
       if (!ok) {  // abort path: let issued copies land
         mbar_drain(q_full, 0);
-        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
-          mbar_drain(kv_full(j % kStages), (uint32_t)((j / kStages) & 1));
+        for (int j = (ik > kStages ? ik - kStages : 0); j < ik; ++j)
+          mbar_drain(k_full(j % kStages), (uint32_t)((j / kStages) & 1));
+        for (int j = (iv > kStages ? iv - kStages : 0); j < iv; ++j)
+          mbar_drain(v_full(j % kStages), (uint32_t)((j / kStages) & 1));
       }
     }
     __syncwarp();
@@ -177,9 +214,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
       tc_fence_after();
       for (int j = 0; j <= n_local && ok; ++j) {
         if (j < n_local) {
-          const int st = j % kStages, sb = j % 2;
-          if (!mbar_wait(kv_full(st), (uint32_t)((j / kStages) & 1), abort_flag, a.err)) { ok = false; break; }
-          if (!mbar_wait(s_free(sb), (uint32_t)((j / 2) & 1) ^ 1u, abort_flag, a.err)) { ok = false; break; }
+          const int st = j % kStages, sb = j % kSBufs;
+          if (!mbar_wait(k_full(st), (uint32_t)((j / kStages) & 1), abort_flag, a.err)) { ok = false; break; }
+          if (!mbar_wait(s_free(sb), (uint32_t)((j / kSBufs) & 1) ^ 1u, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t kbase = sbase + L::kKOff + st * L::kKV;
 #pragma unroll
@@ -192,20 +229,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                       kk >= kSChains ? 1u : 0u);
           }
           umma_commit(s_full(sb));
+          umma_commit(k_empty(st));
         }
         if (j >= 1) {
           const int jp = j - 1, stp = jp % kStages;
-          if (!mbar_wait(p_full, (uint32_t)(jp & 1), abort_flag, a.err)) { ok = false; break; }
+          if (!mbar_wait(p_full(jp & 1), (uint32_t)((jp >> 1) & 1), abort_flag, a.err)) { ok = false; break; }
+          if (!mbar_wait(v_full(stp), (uint32_t)((jp / kStages) & 1), abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t vbase = sbase + L::kVOff + stp * L::kKV;
+          const uint32_t pbase = sbase + L::kPOff + (uint32_t)(jp & 1) * L::kP;
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint64_t ad = sdesc_kmajor_sw128(sbase + L::kPOff + kk * 32);
+            const uint64_t ad = sdesc_kmajor_sw128(pbase + kk * 32);
             const uint64_t bd = sdesc_mnmajor_sw128(vbase + kk * (16 * 128), kBN * 128);
             umma_bf16(tmem + kOCol, ad, bd, idesc_o, (jp > 0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit(pv_done);
-          umma_commit(kv_empty(stp));
+          umma_commit(pv_done(jp & 1));
+          umma_commit(v_empty(stp));
         }
       }
     }
@@ -219,19 +259,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
     bool ok = true;
     uint32_t v[32];
     for (int j = 0; j < n_local; ++j) {
-      const int sb = j % 2;
-      if (!mbar_wait(s_full(sb), (uint32_t)((j / 2) & 1), abort_flag, a.err)) { ok = false; break; }
+      const int sb = j % kSBufs;
+      // waits are made warp-uniform: the warp-wide votes and tcgen05 loads below
+      // need every lane, also on the abort path
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full(sb), (uint32_t)((j / kSBufs) & 1), abort_flag, a.err))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       float s[kBN];
 #pragma unroll
       for (int h = 0; h < kBN / 32; ++h) {
+        // chains summed in a fixed order: ((c0 + c1) + c2) + c3, two loads per wait
+        uint32_t v2[32];
 #pragma unroll
-        for (int ch = 0; ch < kSChains; ++ch) {   // chains summed in a fixed order
+        for (int ch = 0; ch < kSChains; ch += 2) {
           tmem_ld32(lane_base + kSCol + (sb * kSChains + ch) * kBN + h * 32, v);
+          tmem_ld32(lane_base + kSCol + (sb * kSChains + ch + 1) * kBN + h * 32, v2);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            s[h * 32 + e] = (ch == 0) ? __uint_as_float(v[e]) : s[h * 32 + e] + __uint_as_float(v[e]);
+          for (int e = 0; e < 32; ++e) {
+            const float x = (ch == 0) ? __uint_as_float(v[e]) : s[h * 32 + e] + __uint_as_float(v[e]);
+            s[h * 32 + e] = x + __uint_as_float(v2[e]);
+          }
         }
       }
       tc_fence_before();
@@ -246,16 +296,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
         s[e] = (e < valid) ? s[e] * a.scale_log2 : -INFINITY;
         bmax = fmaxf(bmax, s[e]);
       }
-      // P_{j-1} consumed and O up to date before P_j or O is touched
-      if (j >= 1) {
-        if (!mbar_wait(pv_done, (uint32_t)((j - 1) & 1), abort_flag, a.err)) { ok = false; break; }
+      // A row whose block max passes its reference max by the threshold rescales
+      // O; tcgen05.ld/st are warp-wide, so the warp rescales when any lane must
+      // (factor 1 for the others), after every PV so far has finished.  Without
+      // a rescale, P_j only needs its buffer back: PV_{j-2} done.
+      const bool grow = m != -INFINITY && bmax > m + kRescaleThreshold;
+      const bool rescale = __any_sync(0xffffffffu, grow);
+      if (rescale && j >= 1) {
+        if (!__all_sync(0xffffffffu, mbar_wait(pv_done((j - 1) & 1), (uint32_t)(((j - 1) >> 1) & 1),
+                                                abort_flag, a.err))) { ok = false; break; }
+        tc_fence_after();
+      } else if (j >= 2) {
+        if (!__all_sync(0xffffffffu, mbar_wait(pv_done(j & 1), (uint32_t)(((j - 2) >> 1) & 1),
+                                                abort_flag, a.err))) { ok = false; break; }
         tc_fence_after();
       }
-      if (m == -INFINITY) {
-        m = bmax;
-      } else if (bmax > m + kRescaleThreshold) {
-        const float f = exp2f(m - bmax);
-        l *= f;
+      if (rescale) {
+        const float f = grow ? exp2f(m - bmax) : 1.0f;
 #pragma unroll 1
         for (int c0 = 0; c0 < DH; c0 += 32) {
           tmem_ld32(lane_base + kOCol + c0, v);
@@ -265,8 +322,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
           tmem_st32(lane_base + kOCol + c0, v);
         }
         tmem_wait_st();
-        m = bmax;
+        l *= f;
       }
+      if (m == -INFINITY || grow) m = bmax;
       // P = 2^(s - m) as bf16, row r of the K-major swizzled tile
       uint32_t pk[kBN / 2];
 #pragma unroll
@@ -276,7 +334,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
         __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
         pk[e / 2] = *reinterpret_cast<uint32_t*>(&bb);
       }
-      uint8_t* prow = smem + L::kPOff + r * 128;
+      uint8_t* prow = smem + L::kPOff + (j & 1) * L::kP + r * 128;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const int pc = c ^ (r & 7);
@@ -286,10 +344,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(p_full(j & 1));
     }
     // final O, then the partial of this key range
-    if (ok && n_local > 0) ok = mbar_wait(pv_done, (uint32_t)((n_local - 1) & 1), abort_flag, a.err);
+    if (ok && n_local > 0)
+      ok = mbar_wait(pv_done((n_local - 1) & 1), (uint32_t)(((n_local - 1) >> 1) & 1), abort_flag, a.err);
     tc_fence_after();
     const int qr = qt * kRows + r;
     const int rows_total = a.B * a.Hq * a.Tc;

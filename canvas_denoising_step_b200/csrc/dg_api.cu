@@ -260,6 +260,8 @@ int run_dense(dg_ctx* c, int kind, const CUtensorMap& mA, const CUtensorMap& mB,
   a.M = M; a.N = N; a.K = K; a.n_kb = K / 64;
   a.n_tile = c->dense_box;      // one B box per stage covers the activation rows
   a.b_box_rows = c->dense_box;
+  // one 128-row weight slab per tile: pairing two slabs over one activation tile
+  // (dense_pair) measured slower here (6.73 -> 7.30 ms per stack pass)
   a.m_slabs = (M + 127) / 128;
   const int n_chunks = (N + a.n_tile - 1) / a.n_tile;
   a.k_splits = choose_splits(a.m_slabs * n_chunks, a.n_kb, c->num_sms);
