@@ -78,6 +78,7 @@ class OracleConfig:
     rope_enabled: bool = True
     weight_std: float = 0.02
     bf16_weights: bool = True
+    expert_fp8: bool = False     # FP8 E4M3 expert weights, one scale per row (oracle.quant)
     seed: int = 0
 
     @staticmethod
@@ -126,12 +127,20 @@ class LayerWeights:
         """(gate [F,d], up [F,d], down [d,F]) of routed expert e."""
         c = self.cfg
         n = c.d_ff * c.d_model
-        return (self._draw("wg", (c.d_ff, c.d_model), start=e * n),
-                self._draw("wu", (c.d_ff, c.d_model), start=e * n),
-                self._draw("wd", (c.d_model, c.d_ff), start=e * n))
+        return self._lowp((self._draw("wg", (c.d_ff, c.d_model), start=e * n),
+                           self._draw("wu", (c.d_ff, c.d_model), start=e * n),
+                           self._draw("wd", (c.d_model, c.d_ff), start=e * n)))
 
     def shared(self):
-        return self.get("sg"), self.get("su"), self.get("sd")
+        return self._lowp((self.get("sg"), self.get("su"), self.get("sd")))
+
+    def _lowp(self, mats):
+        """The expert weights the layer computes with: as drawn, or (expert_fp8)
+        quantised to FP8 E4M3 with a scale per output row and dequantised."""
+        if not self.cfg.expert_fp8:
+            return mats
+        from .quant import dequantized
+        return tuple(dequantized(m.astype(np.float32)) for m in mats)
 
     # Norm scales are ones under R6.
     def norm(self, _name):

@@ -536,3 +536,66 @@ def test_canvas_step_final_norm_and_embedding_row(monkeypatch):
     assert np.allclose(conf, want, rtol=1e-12)
     # one slot of three commits (k = ceil(3 / 3)); equal confidences -> slot 0
     assert new.tolist() == [[1, 0, 0]] and com.tolist() == [[True, False, False]]
+
+
+# ----------------------------------------------------------------------------- FP8 expert weights
+
+def _e4m3_table():
+    """Every finite E4M3 value, decoded from the format: sign, exponent field e
+    (bias 7), mantissa m; e = 0 gives m * 2^-9, otherwise (1 + m/8) * 2^(e-7);
+    S.1111.111 is NaN.  Returns (values, mantissa parity) of the 254 finite codes."""
+    vals, even = [], []
+    for code in range(256):
+        sgn, e, m = code >> 7, (code >> 3) & 15, code & 7
+        if e == 15 and m == 7:
+            continue
+        v = m * 2.0 ** -9 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7)
+        vals.append(-v if sgn else v)
+        even.append(m % 2 == 0)
+    return np.array(vals), np.array(even)
+
+
+def test_e4m3_rounding_is_the_nearest_code_ties_to_even():
+    from oracle import quant
+    table, even = _e4m3_table()
+    assert table.max() == 448.0 and table[table > 0].min() == 2.0 ** -9
+    x = np.concatenate([RNG.standard_normal(4000) * np.exp(RNG.uniform(-9, 6, 4000)),
+                        (table[np.abs(table) < 448][:-1] + table[np.abs(table) < 448][1:]) / 2])
+    x = np.clip(x, -448, 448).astype(np.float32)
+    got = quant.e4m3_round(x)
+    for xi, gi in zip(x.astype(np.float64), got.astype(np.float64)):
+        d = np.abs(table - xi)
+        best = np.nonzero(d == d.min())[0]
+        if len(best) > 1:                      # a tie: the code with the even mantissa
+            best = [b for b in best if even[b]]
+        assert gi == table[best[0]], (xi, gi, table[best])
+
+
+def test_rowwise_fp8_scale_and_error_bound():
+    from oracle import quant
+    w = (RNG.standard_normal((6, 300)) * 0.02).astype(np.float32)
+    w[2, 7] = -0.2                              # a large entry sets its row's scale
+    w[3] = 0.0                                  # a zero row
+    q, s = quant.e4m3_rowwise(w)
+    amax = np.abs(w).max(axis=1)
+    assert np.array_equal(s, (amax.astype(np.float32) / np.float32(448)).astype(np.float32))
+    assert np.all(np.abs(q) <= 448) and np.all(q[3] == 0) and s[3] == 0
+    assert q[2, 7] == -448.0                    # the row maximum maps to the largest code
+    deq = quant.dequantized(w)
+    # half an E4M3 ulp: relative 2^-4 for normal codes, absolute s * 2^-10 below 2^-6
+    err = np.abs(deq - w.astype(np.float64))
+    bound = np.maximum(np.abs(w) * 2.0 ** -4, s[:, None].astype(np.float64) * 2.0 ** -10)
+    assert np.all(err <= bound * (1 + 1e-6))
+
+
+def test_fp8_experts_are_the_dequantised_drawn_weights():
+    from oracle import quant
+    c16 = tiny_cfg(n_experts=4, d_model=64, d_ff=32)
+    c8 = tiny_cfg(n_experts=4, d_model=64, d_ff=32, expert_fp8=True)
+    W16, W8 = om.layer_weights(c16, 0), om.layer_weights(c8, 0)
+    for a, b in zip(W16.expert(2), W8.expert(2)):
+        assert np.array_equal(b, quant.dequantized(a.astype(np.float32)))
+        assert 0 < np.abs(a - b).max() <= np.abs(a).max() * 2.0 ** -4
+    for a, b in zip(W16.shared(), W8.shared()):
+        assert np.array_equal(b, quant.dequantized(a.astype(np.float32)))
+    assert np.array_equal(W16.get("wq"), W8.get("wq"))     # only the experts change
