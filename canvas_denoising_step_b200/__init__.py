@@ -25,6 +25,8 @@ DG_ERR_CUDA = -4
 DG_ERR_TIMEOUT = -5
 DG_ERR_DEVICE_FAULT = -6
 DG_ERR_UNSUPPORTED = -7
+DG_DTYPE_BF16 = 0
+DG_DTYPE_FP8_E4M3 = 1
 
 
 class DgConfig(ctypes.Structure):
@@ -40,6 +42,7 @@ class DgConfig(ctypes.Structure):
         ("rope_enabled", c_int),
         ("weight_std", c_double),
         ("alloc_limit_bytes", c_size_t),
+        ("expert_dtype", c_int),
     ]
 
 
@@ -108,7 +111,8 @@ def config_from_dict(d: dict, max_batch: int | None = None, max_prompt: int | No
         max_prompt=max_prompt or d["prompt_len"], rms_eps=d["rms_eps"],
         rope_theta=d["rope_theta"], prope_fraction=d["prope_fraction"],
         rope_enabled=int(d["rope_enabled"]), weight_std=d["weight_std"],
-        alloc_limit_bytes=alloc_limit_bytes)
+        alloc_limit_bytes=alloc_limit_bytes,
+        expert_dtype=DG_DTYPE_FP8_E4M3 if d.get("expert_fp8") else DG_DTYPE_BF16)
 
 
 # --------------------------------------------------------------------------- C names

@@ -20,7 +20,11 @@ namespace {
 #define DG_GROUPED_TILE 256
 #endif
 constexpr int kGroupedTile = DG_GROUPED_TILE;   // rows of an expert chunk (B rows per grouped tile)
-constexpr int kGroupedBox = 32;     // B rows per TMA box of a grouped tile
+#ifndef DG_GROUPED_BOX
+#define DG_GROUPED_BOX 64
+#endif
+
+constexpr int kGroupedBox = DG_GROUPED_BOX;   // B rows per TMA box of a grouped tile
 #ifndef DG_DOWN_PAIR
 #define DG_DOWN_PAIR 1
 #endif
@@ -37,6 +41,10 @@ std::string g_create_error;
 
 struct Layer {
   bf16 *wqkv = nullptr, *wo = nullptr, *wr = nullptr, *wgu = nullptr, *wd = nullptr;
+  // FP8 expert weights (expert_dtype = DG_DTYPE_FP8_E4M3): codes and row scales
+  uint8_t *wgu8 = nullptr, *wd8 = nullptr;
+  float *sgu = nullptr, *sd8 = nullptr;
+  CUtensorMap m_gu8, m_d8;
   float *ln_in = nullptr, *ln_post = nullptr, *ln_ff = nullptr;
   CUtensorMap m_qkv, m_o, m_r, m_gu, m_d;
   CUtensorMap m_kp, m_vp;   // prompt K/V of this layer, 64-row boxes
@@ -77,6 +85,7 @@ struct dg_ctx {
   float* w = nullptr;
   uint32_t* bitmap = nullptr;
   int* router_counter = nullptr;
+  int chunk_rows = 0;                // rows of an expert chunk (B rows per grouped tile)
   int* chunk_ready = nullptr;        // per-chunk gate/up -> down hand-over counters
   int n_chunk_ready = 0;
   int32_t* chunk_order = nullptr;    // [n_chunk_ready] the expert chunks longest first
@@ -231,6 +240,8 @@ std::string check_config(const dg_config& c) {
   if (!(c.rms_eps >= 0.f) || !(c.rope_theta > 0.f)) return "rms_eps must be >= 0 and rope_theta > 0";
   if (!(c.prope_fraction >= 0.f && c.prope_fraction <= 1.f)) return "prope_fraction must be in [0, 1]";
   if (!(c.weight_std > 0.0)) return "weight_std must be > 0";
+  if (c.expert_dtype != DG_DTYPE_BF16 && c.expert_dtype != DG_DTYPE_FP8_E4M3)
+    return "expert_dtype must be DG_DTYPE_BF16 or DG_DTYPE_FP8_E4M3";
   // the router groups all rows of a pass in one CTA's shared memory
   if (router_smem_bytes(c.max_batch * c.canvas_len, c.n_experts) >
       (size_t)router_max_smem_bytes())
@@ -279,18 +290,19 @@ int run_dense(dg_ctx* c, int kind, const CUtensorMap& mA, const CUtensorMap& mB,
   return DG_OK;
 }
 
-int run_grouped(dg_ctx* c, int mode, const CUtensorMap& mA, const CUtensorMap& mB, int K, int M,
-                int T) {
+int run_grouped(dg_ctx* c, const Layer& L, int mode, const CUtensorMap& mB, int K, int M) {
   const dg_config& cf = c->cfg;
+  const bool fp8 = L.wgu8 != nullptr;
   GemmArgs a;
   memset(&a, 0, sizeof(a));
   a.mode = mode;
   a.K = K; a.n_kb = K / 64;
   a.M = M;
-  a.n_tile = kGroupedTile;
+  a.n_tile = c->chunk_rows;
   a.b_box_rows = kGroupedBox;
-  // down: 256 weight rows per tile (its H chunk is read once per two slabs)
-  a.pair = mode == GEMM_DOWN && kDownPair ? 1 : 0;
+  // down: 256 weight rows per tile (its H chunk is read once per two slabs); the
+  // FP8-weight GEMMs keep one slab a tile to leave room for their deeper rings
+  a.pair = !fp8 && mode == GEMM_DOWN && kDownPair ? 1 : 0;
   a.m_slabs = a.pair ? (M + 255) / 256 : (M + 127) / 128;
   a.chunk_order = c->chunk_order;
   a.max_chunks = c->n_chunk_ready;
@@ -304,12 +316,29 @@ int run_grouped(dg_ctx* c, int mode, const CUtensorMap& mA, const CUtensorMap& m
   a.err = c->err_dev;
   // gate/up hands each chunk's H rows to down as soon as its slabs are written
   a.chunk_ready = c->chunk_ready;
-  a.ready_target = 4 * ((2 * cf.d_ff + 127) / 128);   // epilogue warps x gate/up slabs
-  (void)T;
-  gemm_plan_smem(a);
-  DG_LAUNCH(c, mode == GEMM_GATEUP ? K_GEMM_GATEUP : K_GEMM_DOWN,
-            gemm_tc_launch(mA, mB, mode == GEMM_GATEUP ? c->m_H_out : c->m_Y_out, a, c->num_sms,
-                           c->stream));
+  a.ready_target = 4 * ((2 * cf.d_ff + 127) / 128);   // epilogue warps x gate/up tiles of a chunk
+  const int kind = mode == GEMM_GATEUP ? K_GEMM_GATEUP : K_GEMM_DOWN;
+  const CUtensorMap& mC = mode == GEMM_GATEUP ? c->m_H_out : c->m_Y_out;
+  if (fp8) {
+    a.w_scale = mode == GEMM_GATEUP ? L.sgu : L.sd8;
+    gemm_fp8_plan_smem(a);
+    DG_LAUNCH(c, kind, gemm_fp8_launch(mode == GEMM_GATEUP ? L.m_gu8 : L.m_d8, mB, mC, a,
+                                       c->num_sms, c->stream));
+  } else {
+    gemm_plan_smem(a);
+    DG_LAUNCH(c, kind, gemm_tc_launch(mode == GEMM_GATEUP ? L.m_gu : L.m_d, mB, mC, a, c->num_sms,
+                                      c->stream));
+  }
+  return DG_OK;
+}
+
+// FP8 codes and row scales of one layer's expert weights, from its bf16 weights.
+int quantize_layer(dg_ctx* c, Layer& L) {
+  if (!L.wgu8) return DG_OK;
+  const dg_config& cf = c->cfg;
+  const long long G = c->G, F = cf.d_ff, d = cf.d_model;
+  DG_CUDA(c, launch_quantize_rows(L.wgu, L.wgu8, L.sgu, G * 2 * F, (int)d, c->stream));
+  DG_CUDA(c, launch_quantize_rows(L.wd, L.wd8, L.sd8, G * d, (int)F, c->stream));
   return DG_OK;
 }
 
@@ -364,7 +393,7 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
     memset(&ra, 0, sizeof(ra));
     ra.logits_in = c->part; ra.splits = splits;
     ra.bias = c->has_bias ? c->router_bias : nullptr;
-    ra.T = T; ra.E = E; ra.k = k; ra.n_shared = cf.n_shared; ra.n_tile = kGroupedTile;
+    ra.T = T; ra.E = E; ra.k = k; ra.n_shared = cf.n_shared; ra.n_tile = c->chunk_rows;
     ra.logits_out = c->router_logits; ra.idx = c->idx; ra.w = c->w;
     ra.bitmap = c->bitmap; ra.counter = c->router_counter;
     ra.offsets_r = c->offsets_r; ra.offsets_g = c->offsets_g; ra.chunk_prefix = c->chunk_prefix;
@@ -376,8 +405,8 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
   DG_LAUNCH(c, K_GATHER, launch_moe_gather(c->xperm, c->perm, T, k, d, c->stream));
 
   // experts (group 0 = shared expert on all rows), SiLU-gated, then down + combine
-  if ((rc = run_grouped(c, GEMM_GATEUP, L.m_gu, c->m_xperm_b, d, 2 * cf.d_ff, T)) != DG_OK) return rc;
-  if ((rc = run_grouped(c, GEMM_DOWN, L.m_d, c->m_H_b, cf.d_ff, d, T)) != DG_OK) return rc;
+  if ((rc = run_grouped(c, L, GEMM_GATEUP, c->m_xperm_b, d, 2 * cf.d_ff)) != DG_OK) return rc;
+  if ((rc = run_grouped(c, L, GEMM_DOWN, c->m_H_b, cf.d_ff, d)) != DG_OK) return rc;
   DG_LAUNCH(c, K_COMBINE, launch_moe_combine(c->Y, c->w, c->inv, T, k, cf.n_shared, d, c->h, w_next,
                                   cf.rms_eps, c->x, c->stream));
   return DG_OK;
@@ -606,6 +635,12 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
     ok &= alloc_n(c, &L.wr, Er * d);
     ok &= alloc_n(c, &L.wgu, (size_t)c->G * 2 * F * d);
     ok &= alloc_n(c, &L.wd, (size_t)c->G * d * F);
+    if (cf.expert_dtype == DG_DTYPE_FP8_E4M3) {
+      ok &= alloc_n(c, &L.wgu8, (size_t)c->G * 2 * F * d);
+      ok &= alloc_n(c, &L.wd8, (size_t)c->G * d * F);
+      ok &= alloc_n(c, &L.sgu, (size_t)c->G * 2 * F);
+      ok &= alloc_n(c, &L.sd8, (size_t)c->G * d);
+    }
     ok &= alloc_n(c, &L.ln_in, d);
     ok &= alloc_n(c, &L.ln_post, d);
     ok &= alloc_n(c, &L.ln_ff, d);
@@ -631,8 +666,9 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
     ok &= alloc_n(c, &c->bitmap, (size_t)E * ((T + 31) / 32));
     ok &= alloc_n(c, &c->router_counter, 4);
     // every expert chunk of a layer: the shared group's plus the routed groups'
-    c->n_chunk_ready = (int)((T + kGroupedTile - 1) / kGroupedTile +
-                             ((size_t)k * T + kGroupedTile - 1) / kGroupedTile + E);
+    c->chunk_rows = kGroupedTile;
+    const size_t cr = (size_t)c->chunk_rows;
+    c->n_chunk_ready = (int)((T + cr - 1) / cr + ((size_t)k * T + cr - 1) / cr + E);
     ok &= alloc_n(c, &c->chunk_ready, (size_t)c->n_chunk_ready);
     ok &= alloc_n(c, &c->chunk_order, (size_t)c->n_chunk_ready);
     ok &= alloc_n(c, &c->tile_counters, 2);
@@ -703,6 +739,10 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
     ok &= make_tmap_2d(&L.m_r, L.wr, d, Er, 128);
     ok &= make_tmap_3d(&L.m_gu, L.wgu, d, 2 * F, c->G, 128);
     ok &= make_tmap_3d(&L.m_d, L.wd, F, d, c->G, 128);
+    if (L.wgu8) {
+      ok &= make_tmap_3d_u8(&L.m_gu8, L.wgu8, d, 2 * F, c->G);
+      ok &= make_tmap_3d_u8(&L.m_d8, L.wd8, F, d, c->G);
+    }
   }
   ok &= make_tmap_2d(&c->m_x_b, c->x, d, Tp, c->dense_box);
   ok &= make_tmap_2d(&c->m_x_a, c->x, d, Tp, 128);
@@ -765,6 +805,8 @@ int dg_init_weights(dg_ctx* c, uint64_t seed) {
     DG_CUDA(c, launch_fill_f32(L.ln_in, d, 1.0f, c->stream));
     DG_CUDA(c, launch_fill_f32(L.ln_post, d, 1.0f, c->stream));
     DG_CUDA(c, launch_fill_f32(L.ln_ff, d, 1.0f, c->stream));
+    int rc = quantize_layer(c, L);
+    if (rc != DG_OK) return rc;
   }
   DG_CUDA(c, cudaStreamSynchronize(c->stream));
   c->weights_ready = true;
@@ -973,6 +1015,7 @@ int dg_load_weights(dg_ctx* c, const char* name, const void* src, size_t bytes) 
   // one contiguous destination, or rows of one bf16 matrix with a row pitch
   void* dst = nullptr;
   size_t n = 0, rows = 0, row_bytes = 0, pitch = 0;
+  Layer* requant_layer = nullptr;
   if (s == "embed") { dst = c->embed; n = V * d * 2; }
   else if (s == "ln_final") { dst = c->ln_final; n = d * 4; }
   else {
@@ -1002,6 +1045,8 @@ int dg_load_weights(dg_ctx* c, const char* name, const void* src, size_t bytes) 
     else return fail(c, DG_ERR_INVALID_ARG, "unknown tensor name");
     if ((base == "sg" || base == "su") && cf.n_shared == 0)
       return fail(c, DG_ERR_INVALID_ARG, "the config has no shared expert");
+    if (base == "wg" || base == "wu" || base == "sg" || base == "su" || base == "wd" || base == "sd")
+      requant_layer = &L;
     if (rows) { row_bytes = d * 2; pitch = 2 * d * 2; n = rows * row_bytes; }
   }
   if (bytes != n) return fail(c, DG_ERR_INVALID_ARG, "byte count does not match the tensor");
@@ -1010,6 +1055,10 @@ int dg_load_weights(dg_ctx* c, const char* name, const void* src, size_t bytes) 
                                  c->stream));
   else
     DG_CUDA(c, cudaMemcpyAsync(dst, src, n, cudaMemcpyDefault, c->stream));
+  if (requant_layer) {   // an expert tensor changed: its FP8 codes follow
+    const int rc = quantize_layer(c, *requant_layer);
+    if (rc != DG_OK) return rc;
+  }
   DG_CUDA(c, cudaStreamSynchronize(c->stream));
   return DG_OK;
 }
@@ -1055,6 +1104,10 @@ int dg_debug_tensor(dg_ctx* c, const char* name, void* dst, size_t bytes, size_t
     else if (base == "wr") { src = L.wr; n = E * d * 2; }
     else if (base == "wgu") { src = L.wgu; n = (size_t)c->G * 2 * F * d * 2; }
     else if (base == "wd") { src = L.wd; n = (size_t)c->G * d * F * 2; }
+    else if (base == "wgu8" && L.wgu8) { src = L.wgu8; n = (size_t)c->G * 2 * F * d; }
+    else if (base == "sgu" && L.sgu) { src = L.sgu; n = (size_t)c->G * 2 * F * 4; }
+    else if (base == "wd8" && L.wd8) { src = L.wd8; n = (size_t)c->G * d * F; }
+    else if (base == "sd8" && L.sd8) { src = L.sd8; n = (size_t)c->G * d * 4; }
     else return fail(c, DG_ERR_INVALID_ARG, "unknown tensor name");
   }
   if (bytes_needed) *bytes_needed = n;

@@ -51,6 +51,8 @@ struct GemmArgs {
   int* tile_counter;
   int max_chunks;
   int pair;
+  const float* w_scale;   // FP8-weight GEMMs: [n_groups][M] fp32 scale of each weight row
+  int sa, sb;             // FP8-weight GEMMs: bf16 A and B ring stages (gemm_fp8_plan_smem)
   int tab_bytes;          // group tables in shared memory (grouped modes)
   int epi_bytes;          // fp32 output staging in shared memory (DENSE, DOWN)
 };
@@ -74,6 +76,19 @@ size_t gemm_smem_bytes(const GemmArgs& a);
 cudaError_t gemm_tc_launch(const CUtensorMap& mapA, const CUtensorMap& mapB,
                            const CUtensorMap& mapC, const GemmArgs& a, int grid,
                            cudaStream_t stream);
+
+// Expert GEMMs with FP8 E4M3 weights (gemm_fp8.cu): GATEUP or DOWN (pair only in
+// DOWN), dynamic tiles (tile_counter and w_scale required).  mapW: the codes
+// [n_groups][M][K] (uint8, boxes 64 codes x 128 rows, make_tmap_3d_u8).
+void gemm_fp8_plan_smem(GemmArgs& a);
+cudaError_t gemm_fp8_launch(const CUtensorMap& mapW, const CUtensorMap& mapB,
+                            const CUtensorMap& mapC, const GemmArgs& a, int grid,
+                            cudaStream_t stream);
+bool make_tmap_3d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid,
+                     uint64_t outer);
+// bf16 rows [rows][K] -> E4M3 codes [rows][K] + fp32 scales [rows] (one per row).
+cudaError_t launch_quantize_rows(const bf16* src, uint8_t* dst, float* scale, long long rows,
+                                 int K, cudaStream_t s);
 
 // ---------------------------------------------------------------- weight init
 // Physical layouts of the generated tensors (see init kernels).

@@ -239,22 +239,32 @@ __global__ void __launch_bounds__(256) eb_commit_kernel(EbCommitArgs a) {
         for (int c = i; c < a.d / 8; c += 256)
           reinterpret_cast<uint4*>(hrow)[c] = reinterpret_cast<const uint4*>(a.hn + t * a.d)[c];
         __syncthreads();
-        const int vid = vb_pick * 256 + i;
-        float e = 0.f;
-        if (vid < a.vocab && vid != a.mask_id) {
-          const uint4* er = reinterpret_cast<const uint4*>(a.embed + (size_t)vid * a.d);
-          float l = 0.f;
-          for (int c = 0; c < a.d / 8; ++c) {
-            const uint4 ev = er[c], hv = reinterpret_cast<const uint4*>(hrow)[c];
-            const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w}, hw[4] = {hv.x, hv.y, hv.z, hv.w};
+        // warp w computes the logits of vocab rows w*32 .. w*32+31 of the block, one
+        // row at a time with the whole warp (coalesced reads of the embedding row,
+        // a fixed-order warp sum); thread i keeps the logit of row i
+        float l_mine = 0.f;
+        const int warp = i >> 5, lane = i & 31;
+        for (int rr = 0; rr < 32; ++rr) {
+          const int vr = vb_pick * 256 + warp * 32 + rr;
+          float part = 0.f;
+          if (vr < a.vocab && vr != a.mask_id) {
+            const uint4* er = reinterpret_cast<const uint4*>(a.embed + (size_t)vr * a.d);
+            for (int c = lane; c < a.d / 8; c += 32) {
+              const uint4 ev = er[c], hv = reinterpret_cast<const uint4*>(hrow)[c];
+              const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w}, hw[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              l = fmaf(__uint_as_float(ew[k] << 16), __uint_as_float(hw[k] << 16), l);
-              l = fmaf(__uint_as_float(ew[k] & 0xFFFF0000u), __uint_as_float(hw[k] & 0xFFFF0000u), l);
+              for (int k = 0; k < 4; ++k) {
+                part = fmaf(__uint_as_float(ew[k] << 16), __uint_as_float(hw[k] << 16), part);
+                part = fmaf(__uint_as_float(ew[k] & 0xFFFF0000u), __uint_as_float(hw[k] & 0xFFFF0000u), part);
+              }
             }
           }
-          e = __expf((l - M) * it);
+          part = warp_sum(part);
+          if (lane == rr) l_mine = part;
         }
+        const int vid = vb_pick * 256 + i;
+        float e = 0.f;
+        if (vid < a.vocab && vid != a.mask_id) e = __expf((l_mine - M) * it);
         const float ci = block_incl_scan(e, s_warp);
         if (i == 0) s_pick = -1;
         __syncthreads();

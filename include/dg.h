@@ -89,7 +89,14 @@ typedef struct dg_config {
   double weight_std;         /* the generator's scale is float32(weight_std * sqrt(3) / 65536) */
   size_t alloc_limit_bytes;  /* 0 = no limit; otherwise dg_create fails with DG_ERR_OOM
                                 instead of allocating more than this many device bytes */
+  int expert_dtype;          /* DG_DTYPE_BF16, or DG_DTYPE_FP8_E4M3: the expert FFN weights
+                                (routed and shared) are used as FP8 E4M3 codes q with one
+                                fp32 scale s per weight row, w = q * s, where
+                                s = max|w_bf16| / 448 and q = E4M3(w_bf16 / s) (fp32
+                                division, round to nearest even); activations stay bf16 */
 } dg_config;
+
+enum { DG_DTYPE_BF16 = 0, DG_DTYPE_FP8_E4M3 = 1 };
 
 /* Pages: "Hands-On with Diffusion Gemma", Detailed Specs (the block structure
  * and sizes a config describes).
@@ -340,6 +347,9 @@ int dg_commit(dg_ctx* ctx, const float* conf, int32_t* canvas, int batch, int st
  *   "wgu:L"    [E+1][2*d_ff][d]   group 0 = shared expert, group g = expert g-1;
  *                                 row 2f = gate row f, row 2f+1 = up row f
  *   "wd:L"     [E+1][d][d_ff]     group 0 = shared expert, group g = expert g-1
+ * with expert_dtype = DG_DTYPE_FP8_E4M3 also the codes and scales:
+ *   "wgu8:L"   uint8 [E+1][2*d_ff][d] (the rows of "wgu:L"), "sgu:L" fp32 [E+1][2*d_ff];
+ *   "wd8:L"    uint8 [E+1][d][d_ff],                          "sd8:L" fp32 [E+1][d]
  * with T = batch * canvas_len rows of the last call. */
 int dg_debug_tensor(dg_ctx* ctx, const char* name, void* dst, size_t bytes,
                     size_t* bytes_needed);

@@ -264,7 +264,14 @@ def _assert_commit_matches_up_to_near_ties(dev_canvas, canvas0, o_logits, mask_i
 
 @pytest.mark.parametrize("name", ["tiny", "ragged"])
 def test_canvas_step_head_and_commit(name):
-    cfg = gpu_cfg(name)
+    canvas_step_check(gpu_cfg(name))
+
+
+def canvas_step_check(cfg):
+    """One pass on the all-mask canvas against the oracle: the head teacher-forced and
+    end to end, the commit bit-exact on the device's confidences and, up to near-ties,
+    equal to the oracle's own pass."""
+    name = cfg["name"]
     c = Ctx(cfg)
     try:
         oc, B, Tc, T = c.oc, c.B, c.Tc, c.T
