@@ -50,7 +50,9 @@ def workload_desc(cfg):
 
 
 def config_json(cfg, n_gpus):
-    return {"workload": workload_desc(cfg), "name": cfg["name"], "batch": cfg["batch"],
+    extra = {"expert_weights": "fp8 e4m3, one fp32 scale per weight row"} if cfg.get("expert_fp8") \
+        else {}
+    return {"workload": workload_desc(cfg), "name": cfg["name"], "batch": cfg["batch"], **extra,
             "canvas_len": cfg["canvas_len"], "prompt_len": cfg["prompt_len"],
             "steps_per_block": cfg["steps"], "n_layers": cfg["n_layers"],
             "l2": "inputs larger than L2: ~50 GB of weights streamed from HBM every step",
@@ -69,7 +71,7 @@ def bytes_per_step(cfg, active_experts=None):
     P, W, L = cfg["prompt_len"], cfg["window"], cfg["n_layers"]
     act = E if active_experts is None else active_experts
     dense = 2 * ((Hq + 2 * Hkv) * dh * d + d * Hq * dh + E * d)
-    experts = 2 * (act + cfg["n_shared"]) * 3 * F * d
+    experts = (act + cfg["n_shared"]) * expert_group_bytes(cfg)
     kv = 0
     for l in range(L):
         vis = P if (l + 1) % cfg["global_every"] == 0 else min(W, P)
@@ -78,13 +80,24 @@ def bytes_per_step(cfg, active_experts=None):
     return L * (dense + experts) + kv + head
 
 
+def expert_group_bytes(cfg, part="all"):
+    """Weight bytes of one expert group: bf16, or (expert_fp8) one byte a code plus a
+    4-byte scale per weight row.  part: "gateup", "down" or "all"."""
+    d, F = cfg["d_model"], cfg["d_ff"]
+    if cfg.get("expert_fp8"):
+        gu, dn = 2 * F * d + 4 * 2 * F, d * F + 4 * d
+    else:
+        gu, dn = 2 * 2 * F * d, 2 * d * F
+    return {"gateup": gu, "down": dn, "all": gu + dn}[part]
+
+
 def gateup_bytes_per_launch(cfg, active_experts=None):
     """Weights of the groups that receive rows, the gathered rows read, H written."""
     d, F, E, k = cfg["d_model"], cfg["d_ff"], cfg["n_experts"], cfg["top_k"]
     act = E if active_experts is None else active_experts
     T = cfg["batch"] * cfg["canvas_len"]
     rows = (k + 1) * T
-    return (act + cfg["n_shared"]) * 2 * F * d * 2 + rows * d * 2 + rows * F * 2
+    return (act + cfg["n_shared"]) * expert_group_bytes(cfg, "gateup") + rows * d * 2 + rows * F * 2
 
 
 def gateup_flops_per_launch(cfg):
@@ -111,7 +124,7 @@ def gateup_roofline(cfg, avg_launch_ms, active_experts, peaks):
     achieved = nbytes / t / 1e9
     return {"bound": "hbm", "kernel": "gemm_gateup", "achieved": achieved, "peak": hbm,
             "unit": "GB/s", "frac": achieved / hbm, "peak_source": kind,
-            "traffic": load_traffic("gemm_gateup") if cfg["name"] == "stack" else None,
+            "traffic": None if cfg.get("expert_fp8") else load_traffic("gemm_gateup", nbytes),
             "algorithmic_bytes_per_launch": nbytes, "avg_launch_ms": avg_launch_ms}
 
 
@@ -142,11 +155,12 @@ def load_peaks():
 
 
 def kernel_src_sha():
-    """Hash of what the GEMM kernel is built from: gemm_tc.cu, dg_common.cuh and
-    the GemmArgs declaration (other declarations in dg_kernels.h do not count)."""
+    """Hash of what the GEMM kernel is built from: gemm_tc.cu, gemm_shared.cuh,
+    dg_common.cuh and the GemmArgs declaration (other declarations in dg_kernels.h
+    do not count)."""
     csrc = os.path.join(ROOT, "canvas_denoising_step_b200", "csrc")
     h = hashlib.sha256()
-    for f in ("gemm_tc.cu", "dg_common.cuh"):
+    for f in ("gemm_tc.cu", "gemm_shared.cuh", "dg_common.cuh"):
         h.update(open(os.path.join(csrc, f), "rb").read())
     hdr = open(os.path.join(csrc, "dg_kernels.h"), "rb").read()
     i = hdr.index(b"struct GemmArgs")
@@ -154,16 +168,17 @@ def kernel_src_sha():
     return h.hexdigest()[:16]
 
 
-def load_traffic(kernel):
-    """DRAM bytes per launch from a committed ncu capture, if it was taken on the
-    current kernel source (else None)."""
+def load_traffic(kernel, algorithmic_bytes):
+    """DRAM bytes per launch: the DRAM / algorithmic byte ratio of a committed ncu
+    capture on a small case (one launch), times this launch's algorithmic bytes;
+    None when the capture was not taken on the current kernel source."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     j = json.load(open(p)).get(kernel)
     if not j or j.get("kernel_src_sha") != kernel_src_sha():
         return None
-    return j.get("dram_bytes_per_launch")
+    return j["dram_over_algorithmic"] * algorithmic_bytes
 
 
 class ClockSampler:
@@ -503,7 +518,7 @@ def layer_bytes(cfg, layer, active_experts):
     P = cfg["prompt_len"]
     vis = P if (layer + 1) % cfg["global_every"] == 0 else min(cfg["window"], P)
     dense = 2 * ((Hq + 2 * Hkv) * dh * d + d * Hq * dh + E * d)
-    return dense + 2 * (active_experts + cfg["n_shared"]) * 3 * F * d + \
+    return dense + (active_experts + cfg["n_shared"]) * expert_group_bytes(cfg) + \
         2 * cfg["batch"] * Hkv * vis * dh * 2
 
 

@@ -30,17 +30,18 @@ def test_gateup_bytes_per_launch_counts_active_groups_rows_and_h():
     assert bench.gateup_bytes_per_launch(cfg) > 1.0e9
 
 
-def test_traffic_is_null_when_the_gemm_sources_changed(tmp_path, monkeypatch):
+def test_traffic_scales_the_captured_ratio_and_is_null_when_the_gemm_sources_changed(
+        tmp_path, monkeypatch):
     prof = tmp_path / "profiles"
     prof.mkdir()
     (prof / "traffic.json").write_text(json.dumps(
-        {"gemm_gateup": {"dram_bytes_per_launch": 123, "kernel_src_sha": "abc"}}))
+        {"gemm_gateup": {"dram_over_algorithmic": 1.25, "kernel_src_sha": "abc"}}))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setattr(bench, "kernel_src_sha", lambda: "abc")
-    assert bench.load_traffic("gemm_gateup") == 123
+    assert bench.load_traffic("gemm_gateup", 400.0) == 500.0
     monkeypatch.setattr(bench, "kernel_src_sha", lambda: "def")
-    assert bench.load_traffic("gemm_gateup") is None
-    assert bench.load_traffic("gemm_down") is None
+    assert bench.load_traffic("gemm_gateup", 400.0) is None
+    assert bench.load_traffic("gemm_down", 400.0) is None
 
 
 def test_clock_sample_stamps_parse():
