@@ -119,6 +119,12 @@ struct dg_ctx {
   float* router_bias = nullptr;
   bool has_bias = false;
   CUtensorMap m_x_b, m_x_a, m_attn_o_b, m_xperm_b, m_H_b, m_x2_b;
+  // half-height B boxes (dense_box / 2 rows) of the two-SM dense projections
+  CUtensorMap m_x_bh, m_attn_o_bh;
+  // Two-SM (cta_group::2) q/k/v, o and bf16 expert GEMMs, when the environment
+  // sets DG_CTA_PAIR=1: co-resident two-CTA clusters, 0 when off.  Measured
+  // slower than the one-SM engine on every workload here, so off by default.
+  int pair_clusters = 0;
   CUtensorMap m_Y_out;   // fp32 expert outputs [1][rows][d], tensor-store map
   CUtensorMap m_H_out;   // bf16 gate/up outputs [rows][F], tensor-store map
   CUtensorMap m_q, m_kc, m_vc;   // attention operands
@@ -262,9 +268,11 @@ int choose_splits(int base_tiles, int n_kb, int num_sms) {
   return best;
 }
 
-// Dense swap-AB projection: part[s][n][m] = X[n] . W[m] over split s.
-int run_dense(dg_ctx* c, int kind, const CUtensorMap& mA, const CUtensorMap& mB, int M, int N,
-              int K, int* splits_out) {
+// Dense swap-AB projection: part[s][n][m] = X[n] . W[m] over split s.  With
+// mB_half (the same activation in half-height boxes) and an even number of
+// weight slabs, tile pairs run on two-SM clusters (gemm_pair.cu).
+int run_dense(dg_ctx* c, int kind, const CUtensorMap& mA, const CUtensorMap& mB,
+              const CUtensorMap* mB_half, int M, int N, int K, int* splits_out) {
   GemmArgs a;
   memset(&a, 0, sizeof(a));
   a.mode = GEMM_DENSE;
@@ -285,7 +293,14 @@ int run_dense(dg_ctx* c, int kind, const CUtensorMap& mA, const CUtensorMap& mB,
   if (!make_tmap_out_f32(&mC, c->part, (uint64_t)M, (uint64_t)N, (uint64_t)a.k_splits))
     return fail(c, DG_ERR_CUDA, "tensor map for a projection output failed");
   const int tiles = a.m_slabs * n_chunks * a.k_splits;
-  DG_LAUNCH(c, kind, gemm_tc_launch(mA, mB, mC, a, std::min(tiles, c->num_sms), c->stream));
+  if (mB_half && c->pair_clusters > 0 && a.m_slabs % 2 == 0) {
+    a.b_box_rows = c->dense_box / 2;
+    gemm_pair_plan_smem(a);
+    DG_LAUNCH(c, kind, gemm_pair_launch(mA, *mB_half, mC, a, std::min(tiles / 2, c->pair_clusters),
+                                        c->stream));
+  } else {
+    DG_LAUNCH(c, kind, gemm_tc_launch(mA, mB, mC, a, std::min(tiles, c->num_sms), c->stream));
+  }
   *splits_out = a.k_splits;
   return DG_OK;
 }
@@ -302,8 +317,12 @@ int run_grouped(dg_ctx* c, const Layer& L, int mode, const CUtensorMap& mB, int 
   a.b_box_rows = kGroupedBox;
   // down: 256 weight rows per tile (its H chunk is read once per two slabs); the
   // FP8-weight GEMMs keep one slab a tile to leave room for their deeper rings
-  a.pair = !fp8 && mode == GEMM_DOWN && kDownPair ? 1 : 0;
+  const bool cta_pair = !fp8 && c->pair_clusters > 0;
+  a.pair = !fp8 && !cta_pair && mode == GEMM_DOWN && kDownPair ? 1 : 0;
   a.m_slabs = a.pair ? (M + 255) / 256 : (M + 127) / 128;
+  // two-SM tiles pair slabs 2p and 2p + 1: an odd slab count gets one empty
+  // slab (its weight rows read as zeros, its outputs are not stored)
+  if (cta_pair) a.m_slabs += a.m_slabs & 1;
   a.chunk_order = c->chunk_order;
   a.max_chunks = c->n_chunk_ready;
   a.tile_counter = c->tile_counters + (mode == GEMM_DOWN ? 1 : 0);
@@ -316,7 +335,9 @@ int run_grouped(dg_ctx* c, const Layer& L, int mode, const CUtensorMap& mB, int 
   a.err = c->err_dev;
   // gate/up hands each chunk's H rows to down as soon as its slabs are written
   a.chunk_ready = c->chunk_ready;
-  a.ready_target = 4 * ((2 * cf.d_ff + 127) / 128);   // epilogue warps x gate/up tiles of a chunk
+  // epilogue warps x gate/up slabs of a chunk (as gate/up counts them)
+  const int gu_slabs = (2 * cf.d_ff + 127) / 128;
+  a.ready_target = 4 * (cta_pair ? gu_slabs + (gu_slabs & 1) : gu_slabs);
   const int kind = mode == GEMM_GATEUP ? K_GEMM_GATEUP : K_GEMM_DOWN;
   const CUtensorMap& mC = mode == GEMM_GATEUP ? c->m_H_out : c->m_Y_out;
   if (fp8) {
@@ -324,6 +345,10 @@ int run_grouped(dg_ctx* c, const Layer& L, int mode, const CUtensorMap& mB, int 
     gemm_fp8_plan_smem(a);
     DG_LAUNCH(c, kind, gemm_fp8_launch(mode == GEMM_GATEUP ? L.m_gu8 : L.m_d8, mB, mC, a,
                                        c->num_sms, c->stream));
+  } else if (cta_pair) {
+    gemm_pair_plan_smem(a);
+    DG_LAUNCH(c, kind, gemm_pair_launch(mode == GEMM_GATEUP ? L.m_gu : L.m_d, mB, mC, a,
+                                        c->pair_clusters, c->stream));
   } else {
     gemm_plan_smem(a);
     DG_LAUNCH(c, kind, gemm_tc_launch(mode == GEMM_GATEUP ? L.m_gu : L.m_d, mB, mC, a, c->num_sms,
@@ -353,7 +378,7 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
   int splits = 1, rc;
 
   // q/k/v projections, RoPE / p-RoPE on the canvas rows
-  if ((rc = run_dense(c, K_GEMM_QKV, L.m_qkv, c->m_x_b, c->NQKV, T, d, &splits)) != DG_OK) return rc;
+  if ((rc = run_dense(c, K_GEMM_QKV, L.m_qkv, c->m_x_b, &c->m_x_bh, c->NQKV, T, d, &splits)) != DG_OK) return rc;
   DG_LAUNCH(c, K_ROPE, launch_qkv_rope(c->part, splits, T, Tc, Hq, Hkv, dh, n_rot_pairs(cf, l), c->rope_cos,
                                c->rope_sin, c->q, c->kc, c->vc, c->stream));
 
@@ -382,12 +407,12 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
   DG_LAUNCH(c, K_ATTN_MERGE, launch_attn_merge(at, c->attn_o, c->stream));
 
   // output projection, post-attention norm + residual, pre-FFN norm
-  if ((rc = run_dense(c, K_GEMM_O, L.m_o, c->m_attn_o_b, d, T, Hq * dh, &splits)) != DG_OK) return rc;
+  if ((rc = run_dense(c, K_GEMM_O, L.m_o, c->m_attn_o_b, &c->m_attn_o_bh, d, T, Hq * dh, &splits)) != DG_OK) return rc;
   DG_LAUNCH(c, K_POST_ATTN, launch_post_attn(c->part, splits, T, d, L.ln_post, L.ln_ff, cf.rms_eps, c->h,
                                 c->xperm, c->stream));
 
   // router
-  if ((rc = run_dense(c, K_GEMM_ROUTER, L.m_r, c->m_x2_b, E, T, d, &splits)) != DG_OK) return rc;
+  if ((rc = run_dense(c, K_GEMM_ROUTER, L.m_r, c->m_x2_b, nullptr, E, T, d, &splits)) != DG_OK) return rc;
   {
     RouterArgs ra;
     memset(&ra, 0, sizeof(ra));
@@ -614,6 +639,10 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
     return fail(nullptr, DG_ERR_UNSUPPORTED, "needs an sm_100 (B200) device");
   }
   c->num_sms = prop.multiProcessorCount;
+  {
+    const char* e = std::getenv("DG_CTA_PAIR");
+    c->pair_clusters = (e && e[0] && e[0] != '0') ? gemm_pair_max_clusters() : 0;
+  }
   const dg_config& cf = c->cfg;
   const int d = cf.d_model, F = cf.d_ff, dh = cf.head_dim, E = cf.n_experts, k = cf.top_k;
   const int Hq = cf.n_q_heads, Hkv = cf.n_kv_heads;
@@ -747,6 +776,8 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
   ok &= make_tmap_2d(&c->m_x_b, c->x, d, Tp, c->dense_box);
   ok &= make_tmap_2d(&c->m_x_a, c->x, d, Tp, 128);
   ok &= make_tmap_2d(&c->m_attn_o_b, c->attn_o, (uint64_t)Hq * dh, Tp, c->dense_box);
+  ok &= make_tmap_2d(&c->m_x_bh, c->x, d, Tp, c->dense_box / 2);
+  ok &= make_tmap_2d(&c->m_attn_o_bh, c->attn_o, (uint64_t)Hq * dh, Tp, c->dense_box / 2);
   ok &= make_tmap_2d(&c->m_xperm_b, c->xperm, d, rows_moe, kGroupedBox);
   ok &= make_tmap_2d(&c->m_x2_b, c->xperm, d, rows_moe, c->dense_box);
   ok &= make_tmap_2d(&c->m_H_b, c->H, F, rows_moe, kGroupedBox);

@@ -34,8 +34,10 @@ struct GemmArgs {
   const float* inv_temp;  // HEAD: NULL, or the inverse temperature (device) for the
   float* head_q;          //   entropy variant, which also writes sum z e^z to head_q
   int* err;
-  // shared-memory and TMEM plan (gemm_plan_smem)
+  // shared-memory and TMEM plan (gemm_plan_smem): stages = k-blocks in flight at
+  // most, stage_bytes = the largest k-block, ring_bytes = the operand ring
   int stages, a_bytes, b_bytes, stage_bytes, b_box_rows;
+  int ring_bytes;
   int n_bufs;
   // Gate/up -> down hand-over without a whole-grid wait: GATEUP adds 1 to
   // chunk_ready[c] per epilogue warp once its H rows of chunk c are written;
@@ -70,6 +72,14 @@ bool make_tmap_f32_sw128(CUtensorMap* map, float* base, uint64_t inner, uint64_t
 bool make_tmap_out_f32(CUtensorMap* map, float* base, uint64_t inner, uint64_t mid,
                        uint64_t outer);
 void gemm_plan_smem(GemmArgs& a);
+// Two-SM (cta_group::2) dense projection: clusters of two CTAs, each holding one
+// 128-row weight slab and half of the tile's activation rows (mapB_half: boxes
+// of b_box_rows = n_tile / 2 rows).  DENSE only, m_slabs even.
+void gemm_pair_plan_smem(GemmArgs& a);
+int gemm_pair_max_clusters();   // co-resident two-CTA clusters of the pair GEMM (0: none)
+cudaError_t gemm_pair_launch(const CUtensorMap& mapA, const CUtensorMap& mapB_half,
+                             const CUtensorMap& mapC, const GemmArgs& a, int clusters,
+                             cudaStream_t stream);
 size_t gemm_smem_bytes(const GemmArgs& a);
 // mapC: the output map (DENSE: fp32 [k_splits][N][M]; DOWN: fp32 [1][rows][M];
 // GATEUP: bf16 H [rows][F]); any valid map for HEAD, which does not use it.
