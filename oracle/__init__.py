@@ -18,8 +18,10 @@ numpy float64.  Each function cites the passage of the pages it follows:
   section "How Text Diffusion Actually Works".
 
 Where those pages are silent the reading taken is stated at the function.
-``eb_sampler`` holds the entropy-bounded denoising rule (the next row of the
-build; its readings are stated in that module).
+``eb_sampler`` holds the entropy-bounded denoising rule and ``encoder`` the
+causal encoder (prompt prefill, context building) with the block-autoregressive
+outer loop (rows of the build after the step itself; their readings are stated
+in those modules).
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (brute force, closed forms, identities and invariants); the end-to-end values
 of a whole step are pinned only through those parts, because the pages print
