@@ -706,6 +706,126 @@ def run_eb_case(args, cfg):
         "gpu_launches": launches * args.steps, "clocks": clk}), flush=True)
 
 
+def encoder_bytes(cfg, active_avg, chunk=None):
+    """Algorithmic HBM bytes of encoding the workload's prompt (dg_encode) in chunks of
+    `chunk` tokens (canvas_len by default): per chunk, every layer's weights the chunk
+    needs once (q/k/v/o,
+    router, the shared expert and `active_avg` routed experts per layer on average),
+    the layer's visible cached K/V once (local layers: the window - 1 positions before
+    the chunk at most) plus the chunk's own K/V appended, and the chunk's embedding rows."""
+    d, E, L, B = cfg["d_model"], cfg["n_experts"], cfg["n_layers"], cfg["batch"]
+    dh, Hq, Hkv = cfg["head_dim"], cfg["n_q_heads"], cfg["n_kv_heads"]
+    P, W = cfg["prompt_len"], cfg["window"]
+    Tc = chunk or cfg["canvas_len"]
+    dense = 2 * ((Hq + 2 * Hkv) * dh * d + d * Hq * dh + E * d)
+    n_chunks, kv = 0, 0
+    for o in range(0, P, Tc):
+        m = min(Tc, P - o)
+        n_chunks += 1
+        for l in range(L):
+            vis = o if (l + 1) % cfg["global_every"] == 0 else min(W - 1, o)
+            kv += 2 * B * Hkv * (vis + m) * dh * 2
+    experts = n_chunks * L * (active_avg + cfg["n_shared"]) * expert_group_bytes(cfg)
+    return n_chunks * L * dense + experts + kv + B * P * d * 2, n_chunks
+
+
+def encoder_flops(cfg):
+    """Algorithmic FLOPs of encoding the workload's prompt: per token and layer the
+    q/k/v, o and router projections, the shared and top-k experts (gate, up, down),
+    and causal attention QK^T and PV over the positions the token sees (all before it
+    and itself on a global layer, the last `window` on a local one)."""
+    d, F, E, k, L, B = (cfg["d_model"], cfg["d_ff"], cfg["n_experts"], cfg["top_k"],
+                        cfg["n_layers"], cfg["batch"])
+    dh, Hq, Hkv, P, W = cfg["head_dim"], cfg["n_q_heads"], cfg["n_kv_heads"], \
+        cfg["prompt_len"], cfg["window"]
+    per_token = 2 * ((Hq + 2 * Hkv) * dh * d + d * Hq * dh + E * d) + \
+        2 * (k + cfg["n_shared"]) * 3 * F * d
+    total = 0
+    for l in range(L):
+        glob = (l + 1) % cfg["global_every"] == 0
+        # sum over positions p of the keys p sees
+        keys = P * (P + 1) // 2 if glob else \
+            sum(min(p + 1, W) for p in range(P)) if P <= 4 * W else \
+            W * (W + 1) // 2 + (P - W) * W
+        total += B * (P * per_token + 2 * 2 * Hq * dh * keys)
+    return total
+
+
+def run_encode_case(args, cfg):
+    """The causal encoder (dg_encode) over the workload's prompt: K encodings of
+    prompt_len seeded random tokens per sequence from an empty context, after W
+    warm-ups.  Reports encoded prompt tokens per second and the encoding against its
+    HBM roofline (encoder_bytes)."""
+    import numpy as np
+    import torch
+    import canvas_denoising_step_b200 as dg
+
+    torch.cuda.set_device(0)
+    stream = torch.cuda.Stream()
+    B, P, L, Tc = cfg["batch"], cfg["prompt_len"], cfg["n_layers"], cfg["canvas_len"]
+    # room for up to 2048 rows a pass (as the batched workload): dg_encode takes chunks
+    # of max_batch * canvas_len / batch tokens, and every chunk reads all the weights
+    mb = max(B, min(2048 // Tc, B * -(-P // Tc)))
+    with torch.cuda.stream(stream):
+        ctx = dg.dg_create(dg.config_from_dict(cfg, max_batch=mb, max_context=P),
+                           stream.cuda_stream)
+        dg.dg_init_weights(ctx, cfg["seed"])
+        g = np.random.default_rng(9)
+        toks = torch.from_numpy(g.integers(1, cfg["vocab"], size=(B, P)).astype(np.int32)).cuda()
+
+        def run(n):
+            for _ in range(n):
+                dg.dg_reset_context(ctx)
+                dg.dg_encode(ctx, toks.data_ptr(), B, P)
+
+        run(args.warmup)
+        act = torch.empty(L, dtype=torch.int32, device="cuda")
+        dg.dg_debug_tensor(ctx, "expert_active", act.data_ptr(), 4 * L)
+        act0 = float(act.sum().item())
+        clocks = ClockSampler(0)
+        clocks.start()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        stream.synchronize()
+        clocks.mark_begin()
+        e0.record(stream)
+        run(args.steps)
+        e1.record(stream)
+        stream.synchronize()
+        clocks.mark_end()
+        clk = clocks.stop()
+        ms = e0.elapsed_time(e1) / args.steps
+        dg.dg_debug_tensor(ctx, "expert_active", act.data_ptr(), 4 * L)
+        chunk = mb * Tc // B
+        n_chunks = -(-P // chunk)
+        active = (float(act.sum().item()) - act0) / (args.steps * n_chunks * L)
+        dg.dg_destroy(ctx)
+    peaks = load_peaks()
+    nbytes, _ = encoder_bytes(cfg, active, chunk)
+    flops = encoder_flops(cfg)
+    hbm, tflops = peaks[0], peaks[1]
+    bytes_ms = nbytes / (hbm * 1e9) * 1e3
+    flops_ms = flops / (tflops * 1e12) * 1e3
+    roof_ms = max(bytes_ms, flops_ms)
+    print(json.dumps({
+        "metric": "encoded prompt tokens/sec on 1 B200 (causal encoder); % of its HBM roofline",
+        "value": B * P / (ms / 1e3), "unit": "prompt tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": dict(config_json(cfg, 1),
+                                            case=f"encode {P} random prompt tokens per sequence "
+                                                 f"in chunks of {chunk}"),
+        "encode_roofline": {"bytes": nbytes, "flops": flops,
+                            "active_experts_per_layer_chunk": active,
+                            "bytes_ms": bytes_ms, "flops_ms": flops_ms, "roofline_ms": roof_ms,
+                            "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
+                            "achieved_tflops": flops / (ms / 1e3) / 1e12,
+                            "frac_of_roofline": roof_ms / ms,
+                            "bound": "tensor" if flops_ms > bytes_ms else "hbm",
+                            "peak": tflops if flops_ms > bytes_ms else hbm,
+                            "peak_source": peaks[2]},
+        "clocks": clk}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -714,8 +834,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["step", "layer"], default="step",
-                    help="step: full canvas passes (the headline); layer: dg_layer_forward")
+    ap.add_argument("--case", choices=["step", "layer", "encode"], default="step",
+                    help="step: full canvas passes (the headline); layer: dg_layer_forward; "
+                         "encode: the causal encoder over the prompt")
     ap.add_argument("--layer", type=int, default=0)
     ap.add_argument("--sampler", choices=["fixed", "eb"], default="fixed",
                     help="fixed: k = ceil(r / steps_left) commits (the headline); eb: "
@@ -730,6 +851,9 @@ def main():
                                          for kv in args.set})
     if args.case == "layer":
         run_layer_case(args, cfg)
+        return
+    if args.case == "encode":
+        run_encode_case(args, cfg)
         return
     if args.sampler == "eb":
         run_eb_case(args, cfg)

@@ -43,6 +43,7 @@ class DgConfig(ctypes.Structure):
         ("weight_std", c_double),
         ("alloc_limit_bytes", c_size_t),
         ("expert_dtype", c_int),
+        ("max_context", c_int),
     ]
 
 
@@ -67,6 +68,11 @@ _SIGS = {
     "dg_canvas_step": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p]),
     "dg_canvas_step_host": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p]),
     "dg_denoise_block": (c_int, [c_void_p, c_void_p, c_int, c_int]),
+    "dg_encode": (c_int, [c_void_p, c_void_p, c_int, c_int]),
+    "dg_reset_context": (c_int, [c_void_p]),
+    "dg_context_length": (c_int, [c_void_p, POINTER(c_int)]),
+    "dg_context_kv": (c_int, [c_void_p, c_int, c_void_p, c_void_p]),
+    "dg_generate": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p]),
     "dg_eb_step": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
                            c_void_p]),
     "dg_eb_denoise_block": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p]),
@@ -100,7 +106,7 @@ def _check(ctx, code: int, func: str):
 
 
 def config_from_dict(d: dict, max_batch: int | None = None, max_prompt: int | None = None,
-                     alloc_limit_bytes: int = 0) -> DgConfig:
+                     alloc_limit_bytes: int = 0, max_context: int = 0) -> DgConfig:
     """A DgConfig from a workload description (the keys of synth.CONFIGS)."""
     return DgConfig(
         n_layers=d["n_layers"], d_model=d["d_model"], n_q_heads=d["n_q_heads"],
@@ -112,7 +118,8 @@ def config_from_dict(d: dict, max_batch: int | None = None, max_prompt: int | No
         rope_theta=d["rope_theta"], prope_fraction=d["prope_fraction"],
         rope_enabled=int(d["rope_enabled"]), weight_std=d["weight_std"],
         alloc_limit_bytes=alloc_limit_bytes,
-        expert_dtype=DG_DTYPE_FP8_E4M3 if d.get("expert_fp8") else DG_DTYPE_BF16)
+        expert_dtype=DG_DTYPE_FP8_E4M3 if d.get("expert_fp8") else DG_DTYPE_BF16,
+        max_context=max_context)
 
 
 # --------------------------------------------------------------------------- C names
@@ -153,6 +160,30 @@ def dg_canvas_step_host(ctx: int, canvas_host: int, batch: int, steps_left: int,
 
 def dg_denoise_block(ctx: int, canvas: int, batch: int, n_steps: int) -> None:
     _check(ctx, _lib.dg_denoise_block(ctx, canvas, batch, n_steps), "dg_denoise_block")
+
+
+def dg_encode(ctx: int, tokens: int, batch: int, n: int) -> None:
+    _check(ctx, _lib.dg_encode(ctx, tokens, batch, n), "dg_encode")
+
+
+def dg_reset_context(ctx: int) -> None:
+    _check(ctx, _lib.dg_reset_context(ctx), "dg_reset_context")
+
+
+def dg_context_length(ctx: int) -> int:
+    n = c_int()
+    _check(ctx, _lib.dg_context_length(ctx, ctypes.byref(n)), "dg_context_length")
+    return n.value
+
+
+def dg_context_kv(ctx: int, layer: int, k_out: int, v_out: int) -> None:
+    _check(ctx, _lib.dg_context_kv(ctx, layer, k_out, v_out), "dg_context_kv")
+
+
+def dg_generate(ctx: int, prompt: int, batch: int, n_prompt: int, n_blocks: int, n_steps: int,
+                out: int) -> None:
+    _check(ctx, _lib.dg_generate(ctx, prompt, batch, n_prompt, n_blocks, n_steps, out),
+           "dg_generate")
 
 
 def dg_eb_step(ctx: int, canvas: int, batch: int, step: int, n_max: int, u: int,

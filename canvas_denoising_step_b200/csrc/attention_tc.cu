@@ -23,6 +23,8 @@
 //                    128-byte-swizzle layout the MMA reads.
 // The CTA writes the un-normalised partial (O, m, l) of its key range; the
 // log-sum-exp merge kernel combines the ranges.
+#include <climits>
+
 #include "dg_kernels.h"
 
 namespace dg {
@@ -86,8 +88,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
   const int nbp = (a.n_vis + kBN - 1) / kBN;            // prompt-key blocks
   const int nbc = (a.Tc + kBN - 1) / kBN;               // canvas-key blocks
   const int nb = nbp + nbc;
-  const int jb0 = (int)(((long long)chunk * nb) / a.n_chunks);
-  const int jb1 = (int)(((long long)(chunk + 1) * nb) / a.n_chunks);
+  // Key blocks this query tile needs: all of them, or in causal mode those that
+  // meet some row's visible positions [P + i - window + 1, P + i] (the tile's rows
+  // are new tokens i_min .. i_max, or every i when the tile crosses a head).
+  int js = 0, je = nb;
+  if (a.causal) {
+    const int r0 = qt * kRows, r1 = min(r0 + kRows, q_rows) - 1;
+    const int i_min = (r0 / a.Tc == r1 / a.Tc) ? r0 % a.Tc : 0;
+    const int i_max = (r0 / a.Tc == r1 / a.Tc) ? r1 % a.Tc : a.Tc - 1;
+    je = nbp + i_max / kBN + 1;
+    if (a.window > 0) {
+      const int lo = a.P + i_min - a.window + 1;        // lowest position a row sees
+      const int first = a.P - a.n_vis;                  // position of prompt block 0, key 0
+      js = (lo < a.P) ? max(0, lo - first) / kBN : nbp + (lo - a.P) / kBN;
+    }
+  }
+  const int jb0 = js + (int)(((long long)chunk * (je - js)) / a.n_chunks);
+  const int jb1 = js + (int)(((long long)(chunk + 1) * (je - js)) / a.n_chunks);
   const int n_local = jb1 - jb0;
   // TMEM: O at [0, DH); then two S buffers (the next QK^T runs while the
   // softmax reads the last one), each split into two independent accumulator
@@ -135,7 +152,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
     const int jg = jb0 + j;
     if (jg < nbp) {
       mk = &mapKp; mv = &mapVp;
-      row = (b * a.Hkv + g) * a.P + (a.P - a.n_vis) + jg * kBN;
+      row = (b * a.Hkv + g) * a.kv_stride + (a.P - a.n_vis) + jg * kBN;
     } else {
       mk = &mapKc; mv = &mapVc;
       row = (b * a.Hkv + g) * a.Tc + (jg - nbp) * kBN;
@@ -255,6 +272,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
     const int q = warp & 3;
     const int r = q * 32 + lane;                       // query row in the tile
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    // causal mode: this row's new-token index i and its visible positions
+    // [lo_pos, P + i] (keys are numbered by position: cached ones from P - n_vis)
+    const int i_row = (qt * kRows + r) % a.Tc;
+    const int hi_pos = a.P + i_row;
+    const int lo_pos = a.window > 0 ? hi_pos - a.window + 1 : INT_MIN;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     uint32_t v[32];
@@ -291,10 +313,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
       const int jg = jb0 + j;
       const int valid = (jg < nbp) ? min(kBN, a.n_vis - jg * kBN) : min(kBN, a.Tc - (jg - nbp) * kBN);
       float bmax = -INFINITY;
+      if (a.causal) {
+        const int pos0 = (jg < nbp) ? a.P - a.n_vis + jg * kBN : a.P + (jg - nbp) * kBN;
 #pragma unroll
-      for (int e = 0; e < kBN; ++e) {
-        s[e] = (e < valid) ? s[e] * a.scale_log2 : -INFINITY;
-        bmax = fmaxf(bmax, s[e]);
+        for (int e = 0; e < kBN; ++e) {
+          const bool vis = e < valid && pos0 + e <= hi_pos && pos0 + e >= lo_pos;
+          s[e] = vis ? s[e] * a.scale_log2 : -INFINITY;
+          bmax = fmaxf(bmax, s[e]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < kBN; ++e) {
+          s[e] = (e < valid) ? s[e] * a.scale_log2 : -INFINITY;
+          bmax = fmaxf(bmax, s[e]);
+        }
       }
       // A row whose block max passes its reference max by the threshold rescales
       // O; tcgen05.ld/st are warp-wide, so the warp rescales when any lane must
@@ -325,11 +357,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
         l *= f;
       }
       if (m == -INFINITY || grow) m = bmax;
-      // P = 2^(s - m) as bf16, row r of the K-major swizzled tile
+      // P = 2^(s - m) as bf16, row r of the K-major swizzled tile (a row that has
+      // seen no visible key yet, possible in causal mode, writes zeros)
+      const float msub = (m == -INFINITY) ? 0.f : m;
       uint32_t pk[kBN / 2];
 #pragma unroll
       for (int e = 0; e < kBN; e += 2) {
-        const float p0 = exp2f(s[e] - m), p1 = exp2f(s[e + 1] - m);
+        const float p0 = exp2f(s[e] - msub), p1 = exp2f(s[e + 1] - msub);
         l += p0 + p1;
         __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
         pk[e / 2] = *reinterpret_cast<uint32_t*>(&bb);

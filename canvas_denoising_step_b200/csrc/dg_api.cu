@@ -51,6 +51,9 @@ struct Layer {
   const bf16* kp = nullptr;
   const bf16* vp = nullptr;
   int kv_batch = 0, kv_P = 0;
+  int kv_stride = 0;   // rows per (sequence, kv head) behind m_kp / m_vp
+  // the library's own KV cache (max_context > 0): [max_batch][Hkv][max_context][dh]
+  bf16 *own_k = nullptr, *own_v = nullptr;
 };
 
 }  // namespace
@@ -125,6 +128,10 @@ struct dg_ctx {
   // sets DG_CTA_PAIR=1: co-resident two-CTA clusters, 0 when off.  Measured
   // slower than the one-SM engine on every workload here, so off by default.
   int pair_clusters = 0;
+  // Encoded context in the library's own KV cache (dg_encode / dg_generate):
+  // positions held, and the batch they belong to (0: none yet).
+  int ctx_len = 0, ctx_batch = 0;
+  int32_t* gen_canvas = nullptr;   // [max_batch][canvas_len] working canvas of dg_generate
   CUtensorMap m_Y_out;   // fp32 expert outputs [1][rows][d], tensor-store map
   CUtensorMap m_H_out;   // bf16 gate/up outputs [rows][F], tensor-store map
   CUtensorMap m_q, m_kc, m_vc;   // attention operands
@@ -167,12 +174,12 @@ int fail(dg_ctx* c, int code, const std::string& msg) {
 enum KernelKind {
   K_EMBED, K_ROPE_TABLE, K_GEMM_QKV, K_ROPE, K_ATTN, K_ATTN_MERGE, K_GEMM_O, K_POST_ATTN,
   K_GEMM_ROUTER, K_ROUTER, K_GATHER, K_GEMM_GATEUP, K_GEMM_DOWN, K_COMBINE,
-  K_GEMM_HEAD, K_HEAD_MERGE, K_COMMIT, K_NUM_KINDS
+  K_GEMM_HEAD, K_HEAD_MERGE, K_COMMIT, K_KV_APPEND, K_NUM_KINDS
 };
 const char* const kKindNames[K_NUM_KINDS] = {
   "embed_norm", "rope_table", "gemm_qkv", "qkv_rope", "attention", "attn_merge", "gemm_o",
   "post_attn", "gemm_router", "router", "moe_gather", "gemm_gateup",
-  "gemm_down", "moe_combine", "gemm_head", "head_merge", "commit"};
+  "gemm_down", "moe_combine", "gemm_head", "head_merge", "commit", "kv_append"};
 
 // Per-launch CUDA events while profiling is on (events come from a growing pool).
 int prof_begin(dg_ctx* c, int kind) {
@@ -241,6 +248,7 @@ std::string check_config(const dg_config& c) {
   if (c.canvas_len < 1 || c.canvas_len > 256) return "canvas_len must be in [1, 256]";
   if (c.max_batch < 1 || (long long)c.max_batch * c.canvas_len > 4096) return "max_batch * canvas_len must be in [1, 4096]";
   if (c.max_prompt < 1) return "max_prompt must be >= 1";
+  if (c.max_context < 0) return "max_context must be >= 0";
   if (c.mask_id < 0 || c.mask_id >= c.vocab) return "mask_id must be in [0, vocab)";
   if (c.window < 1 || c.global_every < 1) return "window and global_every must be >= 1";
   if (!(c.rms_eps >= 0.f) || !(c.rope_theta > 0.f)) return "rms_eps must be >= 0 and rope_theta > 0";
@@ -367,12 +375,16 @@ int quantize_layer(dg_ctx* c, Layer& L) {
   return DG_OK;
 }
 
-// One decoder block on c->h / c->x (x = input-normed h).  On return h is the
-// block output and x = bf16(rmsnorm(h) * w_next) (or bf16(h) when w_next is NULL).
-int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
+// One block on c->h / c->x (x = input-normed h) for B sequences of Tc rows.  On
+// return h is the block output and x = bf16(rmsnorm(h) * w_next) (or bf16(h)
+// when w_next is NULL).  The decoder (causal false) attends jointly over the
+// visible prompt keys and all Tc canvas keys; the encoder (causal true) attends
+// causally over the cached positions and the Tc new tokens, then appends the
+// new tokens' keys and values to the layer's own cache at positions P ...
+int run_layer(dg_ctx* c, int l, int B, const float* w_next, int Tc, bool causal) {
   const dg_config& cf = c->cfg;
   Layer& L = c->layers[l];
-  const int Tc = cf.canvas_len, T = B * Tc, d = cf.d_model, dh = cf.head_dim;
+  const int T = B * Tc, d = cf.d_model, dh = cf.head_dim;
   const int Hq = cf.n_q_heads, Hkv = cf.n_kv_heads, E = cf.n_experts, k = cf.top_k;
   const int P = L.kv_P;
   int splits = 1, rc;
@@ -386,7 +398,15 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
   AttnTcArgs ta;
   memset(&ta, 0, sizeof(ta));
   ta.B = B; ta.Hq = Hq; ta.Hkv = Hkv; ta.Tc = Tc; ta.P = P; ta.dh = dh;
-  ta.n_vis = is_global(cf, l) ? P : std::min(cf.window, P);
+  ta.kv_stride = L.kv_stride;
+  if (!causal) {
+    ta.n_vis = is_global(cf, l) ? P : std::min(cf.window, P);
+  } else {
+    // new token 0 (position P) sees the last window - 1 cached positions
+    ta.causal = 1;
+    ta.window = is_global(cf, l) ? 0 : cf.window;
+    ta.n_vis = is_global(cf, l) ? P : std::min(cf.window - 1, P);
+  }
   {
     // key-block ranges per (canvas, kv head, query tile): about one CTA per SM
     const int nb = attn_tc_blocks(ta.n_vis, Tc);
@@ -405,6 +425,9 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next) {
   at.n_chunks = ta.n_chunks;
   at.part_o = c->attn_po; at.part_ml = c->attn_ml;
   DG_LAUNCH(c, K_ATTN_MERGE, launch_attn_merge(at, c->attn_o, c->stream));
+  if (causal)
+    DG_LAUNCH(c, K_KV_APPEND, launch_kv_append(c->kc, c->vc, L.own_k, L.own_v, B, Hkv, Tc, dh,
+                                               cf.max_context, P, c->stream));
 
   // output projection, post-attention norm + residual, pre-FFN norm
   if ((rc = run_dense(c, K_GEMM_O, L.m_o, c->m_attn_o_b, &c->m_attn_o_bh, d, T, Hq * dh, &splits)) != DG_OK) return rc;
@@ -454,7 +477,8 @@ int check_prompt_state(dg_ctx* c, int batch) {
 
 int ensure_rope(dg_ctx* c, int P) {
   if (c->rope_P != P) {
-    DG_LAUNCH(c, K_ROPE_TABLE, launch_rope_table(c->rope_cos, c->rope_sin, c->cfg.canvas_len,
+    // positions P .. P + Tmax - 1: a canvas, or an encoder chunk of up to Tmax rows
+    DG_LAUNCH(c, K_ROPE_TABLE, launch_rope_table(c->rope_cos, c->rope_sin, c->Tmax,
                                    c->cfg.head_dim / 2, P, (double)c->cfg.rope_theta, c->stream));
     c->rope_P = P;
   }
@@ -476,7 +500,7 @@ int record_step(dg_ctx* c, int B, bool eb) {
                                  c->stream));
   for (int l = 0; l < cf.n_layers; ++l) {
     const float* w_next = (l + 1 < cf.n_layers) ? c->layers[l + 1].ln_in : c->ln_final;
-    if ((rc = run_layer(c, l, B, w_next)) != DG_OK) return rc;
+    if ((rc = run_layer(c, l, B, w_next, cf.canvas_len, false)) != DG_OK) return rc;
   }
   // tied vocab head with the fused (max, argmax, sum-exp) reduction
   GemmArgs a;
@@ -611,6 +635,67 @@ int read_device_error(dg_ctx* c) {
   return DG_OK;
 }
 
+// Point every layer's prompt K/V at the library's own cache: batch B, the
+// positions encoded so far (ctx_len), rows max_context apart.
+int use_own_cache(dg_ctx* c, int B) {
+  const dg_config& cf = c->cfg;
+  for (auto& L : c->layers) {
+    if (L.kp != L.own_k || L.kv_batch != B || L.kv_P != c->ctx_len) drop_graphs(c);
+    if (L.kp != L.own_k || L.kv_batch != B) {
+      const uint64_t rows = (uint64_t)B * cf.n_kv_heads * cf.max_context;
+      if (!make_tmap_2d(&L.m_kp, L.own_k, cf.head_dim, rows, 64) ||
+          !make_tmap_2d(&L.m_vp, L.own_v, cf.head_dim, rows, 64))
+        return fail(c, DG_ERR_CUDA, "tensor map for the context K/V failed");
+    }
+    L.kp = L.own_k;
+    L.vp = L.own_v;
+    L.kv_batch = B;
+    L.kv_P = c->ctx_len;
+    L.kv_stride = cf.max_context;
+  }
+  return DG_OK;
+}
+
+// The causal encoder over n tokens per sequence (device or host int32 [B][n],
+// row stride ld), in chunks of up to Tmax / B tokens (the rows a pass over
+// max_batch canvases holds): each chunk's keys and values are appended to the
+// own cache after the positions already held.  Every chunk reads all the
+// layers' weights once, so the longer the chunk the fewer weight bytes a token.
+int encode_tokens(dg_ctx* c, const int32_t* tokens, int B, int n, int ld) {
+  const dg_config& cf = c->cfg;
+  const int chunk = std::max(1, c->Tmax / B);
+  int rc;
+  for (int o = 0; o < n; o += chunk) {
+    const int m = std::min(chunk, n - o);
+    if ((rc = use_own_cache(c, B)) != DG_OK) return rc;
+    if ((rc = ensure_rope(c, c->ctx_len)) != DG_OK) return rc;
+    DG_CUDA(c, cudaMemcpy2DAsync(c->canvas_dev, (size_t)m * 4, tokens + o, (size_t)ld * 4,
+                                 (size_t)m * 4, B, cudaMemcpyDefault, c->stream));
+    DG_LAUNCH(c, K_EMBED, launch_embed_norm(c->canvas_dev, c->embed, nullptr, cf.vocab, B * m,
+                                            cf.d_model, c->layers[0].ln_in, cf.rms_eps, c->h,
+                                            c->x, c->err_dev, c->stream));
+    for (int l = 0; l < cf.n_layers; ++l) {
+      const float* w_next = (l + 1 < cf.n_layers) ? c->layers[l + 1].ln_in : c->ln_final;
+      if ((rc = run_layer(c, l, B, w_next, m, true)) != DG_OK) return rc;
+    }
+    c->ctx_len += m;
+    c->ctx_batch = B;
+  }
+  return DG_OK;
+}
+
+int check_context_args(dg_ctx* c, int batch, int n) {
+  if (c->cfg.max_context < 1)
+    return fail(c, DG_ERR_BAD_STATE, "the context needs dg_config.max_context > 0");
+  if (!c->weights_ready) return fail(c, DG_ERR_BAD_STATE, "weights not initialised");
+  if (batch < 1 || batch > c->cfg.max_batch) return fail(c, DG_ERR_INVALID_ARG, "batch out of range");
+  if (c->ctx_len > 0 && batch != c->ctx_batch)
+    return fail(c, DG_ERR_INVALID_ARG, "batch differs from the batch of the encoded context");
+  if (n < 0 || (long long)c->ctx_len + n > c->cfg.max_context)
+    return fail(c, DG_ERR_INVALID_ARG, "the context would exceed max_context");
+  return DG_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -662,6 +747,11 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
     ok &= alloc_n(c, &L.wqkv, (size_t)c->NQKV * d);
     ok &= alloc_n(c, &L.wo, (size_t)d * Hq * dh);
     ok &= alloc_n(c, &L.wr, Er * d);
+    if (cf.max_context > 0) {
+      const size_t cap = (size_t)cf.max_batch * Hkv * cf.max_context * dh;
+      ok &= alloc_n(c, &L.own_k, cap);
+      ok &= alloc_n(c, &L.own_v, cap);
+    }
     ok &= alloc_n(c, &L.wgu, (size_t)c->G * 2 * F * d);
     ok &= alloc_n(c, &L.wd, (size_t)c->G * d * F);
     if (cf.expert_dtype == DG_DTYPE_FP8_E4M3) {
@@ -727,11 +817,12 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
     ok &= alloc_n(c, &c->eb_last, 4);
     ok &= alloc_n(c, &c->tok, T);
     ok &= alloc_n(c, &c->canvas_dev, T);
+    if (cf.max_context > 0) ok &= alloc_n(c, &c->gen_canvas, T);
     ok &= alloc_n(c, &c->committed_dev, T);
     ok &= alloc_n(c, &c->err_dev, 4);
     ok &= alloc_n(c, &c->expert_active, cf.n_layers);
-    ok &= alloc_n(c, &c->rope_cos, (size_t)cf.canvas_len * dh / 2);
-    ok &= alloc_n(c, &c->rope_sin, (size_t)cf.canvas_len * dh / 2);
+    ok &= alloc_n(c, &c->rope_cos, (size_t)c->Tmax * dh / 2);
+    ok &= alloc_n(c, &c->rope_sin, (size_t)c->Tmax * dh / 2);
     ok &= alloc_n(c, &c->router_bias, E);
   }
   if (!ok) {
@@ -865,6 +956,49 @@ int dg_set_prompt_kv(dg_ctx* c, int layer, const void* k, const void* v, int bat
   L.vp = static_cast<const bf16*>(v);
   L.kv_batch = batch;
   L.kv_P = n_prompt;
+  L.kv_stride = n_prompt;
+  return DG_OK;
+}
+
+int dg_encode(dg_ctx* c, const int32_t* tokens, int batch, int n) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (!tokens) return fail(c, DG_ERR_INVALID_ARG, "null tokens");
+  if (n < 1) return fail(c, DG_ERR_INVALID_ARG, "n must be >= 1");
+  int rc = check_context_args(c, batch, n);
+  if (rc != DG_OK) return rc;
+  if ((rc = encode_tokens(c, tokens, batch, n, n)) != DG_OK) return rc;
+  if ((rc = use_own_cache(c, batch)) != DG_OK) return rc;
+  return read_device_error(c);
+}
+
+int dg_reset_context(dg_ctx* c) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  c->ctx_len = 0;
+  c->ctx_batch = 0;
+  return DG_OK;
+}
+
+int dg_context_length(dg_ctx* c, int* n_out) {
+  if (!c || !n_out) return DG_ERR_INVALID_ARG;
+  *n_out = c->ctx_len;
+  return DG_OK;
+}
+
+int dg_context_kv(dg_ctx* c, int layer, void* k_out, void* v_out) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= c->cfg.n_layers) return fail(c, DG_ERR_INVALID_ARG, "layer out of range");
+  if (!k_out || !v_out) return fail(c, DG_ERR_INVALID_ARG, "null output");
+  if (c->cfg.max_context < 1 || c->ctx_len == 0)
+    return fail(c, DG_ERR_BAD_STATE, "no encoded context");
+  const dg_config& cf = c->cfg;
+  const Layer& L = c->layers[layer];
+  const size_t row = (size_t)cf.head_dim * 2;
+  const int seqs = c->ctx_batch * cf.n_kv_heads;
+  DG_CUDA(c, cudaMemcpy2DAsync(k_out, c->ctx_len * row, L.own_k, (size_t)cf.max_context * row,
+                               c->ctx_len * row, seqs, cudaMemcpyDefault, c->stream));
+  DG_CUDA(c, cudaMemcpy2DAsync(v_out, c->ctx_len * row, L.own_v, (size_t)cf.max_context * row,
+                               c->ctx_len * row, seqs, cudaMemcpyDefault, c->stream));
+  DG_CUDA(c, cudaStreamSynchronize(c->stream));
   return DG_OK;
 }
 
@@ -919,6 +1053,35 @@ int dg_denoise_block(dg_ctx* c, int32_t* canvas, int batch, int n_steps) {
   for (int s = 0; s < n_steps; ++s)
     if ((rc = run_step(c, batch, n_steps - s)) != DG_OK) return rc;
   DG_CUDA(c, cudaMemcpyAsync(canvas, c->canvas_dev, T * 4, cudaMemcpyDefault, c->stream));
+  return read_device_error(c);
+}
+
+int dg_generate(dg_ctx* c, const int32_t* prompt, int batch, int n_prompt, int n_blocks,
+                int n_steps, int32_t* out) {
+  if (!c) return DG_ERR_INVALID_ARG;
+  if (!prompt || !out) return fail(c, DG_ERR_INVALID_ARG, "null prompt or output");
+  if (n_prompt < 1 || n_blocks < 1 || n_steps < 1)
+    return fail(c, DG_ERR_INVALID_ARG, "n_prompt, n_blocks and n_steps must be >= 1");
+  const dg_config& cf = c->cfg;
+  const int Tc = cf.canvas_len;
+  dg_reset_context(c);
+  int rc = check_context_args(c, batch, n_prompt + n_blocks * Tc);
+  if (rc != DG_OK) return rc;
+  if ((rc = encode_tokens(c, prompt, batch, n_prompt, n_prompt)) != DG_OK) return rc;
+  const std::vector<int32_t> mask((size_t)batch * Tc, cf.mask_id);
+  const size_t row_out = (size_t)n_blocks * Tc * 4;
+  for (int blk = 0; blk < n_blocks; ++blk) {
+    // an all-mask canvas denoised against the context, then encoded onto it
+    if ((rc = use_own_cache(c, batch)) != DG_OK) return rc;
+    DG_CUDA(c, cudaMemcpyAsync(c->gen_canvas, mask.data(), mask.size() * 4, cudaMemcpyHostToDevice,
+                               c->stream));
+    if ((rc = dg_denoise_block(c, c->gen_canvas, batch, n_steps)) != DG_OK) return rc;
+    DG_CUDA(c, cudaMemcpy2DAsync(out + (size_t)blk * Tc, row_out, c->gen_canvas, (size_t)Tc * 4,
+                                 (size_t)Tc * 4, batch, cudaMemcpyDefault, c->stream));
+    if ((rc = encode_tokens(c, c->gen_canvas, batch, Tc, Tc)) != DG_OK) return rc;
+  }
+  if ((rc = use_own_cache(c, batch)) != DG_OK) return rc;
+  DG_CUDA(c, cudaStreamSynchronize(c->stream));
   return read_device_error(c);
 }
 
@@ -999,7 +1162,7 @@ int dg_layer_forward(dg_ctx* c, int layer, const void* x_in, void* x_out, int n_
   DG_LAUNCH(c, K_EMBED, launch_embed_norm(nullptr, nullptr, static_cast<const bf16*>(x_in), c->cfg.vocab,
                                  n_rows, d, L.ln_in, c->cfg.rms_eps, c->h, c->x, c->err_dev,
                                  c->stream));
-  if ((rc = run_layer(c, layer, B, nullptr)) != DG_OK) return rc;
+  if ((rc = run_layer(c, layer, B, nullptr, c->cfg.canvas_len, false)) != DG_OK) return rc;
   DG_CUDA(c, cudaMemcpyAsync(x_out, c->x, (size_t)n_rows * d * 2, cudaMemcpyDeviceToDevice,
                              c->stream));
   c->last_T = n_rows;

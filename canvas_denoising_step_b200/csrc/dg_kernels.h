@@ -125,6 +125,9 @@ unsigned long long stream_key_host(unsigned long long seed, unsigned long long t
 cudaError_t launch_init(const InitArgs& a, cudaStream_t s);
 cudaError_t launch_fill_f32(float* p, long long n, float v, cudaStream_t s);
 cudaError_t launch_set_int(int* p, int v, cudaStream_t s);
+// kc / vc [B][Hkv][n][dh] -> cache [B][Hkv][C][dh] at positions P0 .. P0 + n - 1.
+cudaError_t launch_kv_append(const bf16* kc, const bf16* vc, bf16* ck, bf16* cv, int B, int Hkv,
+                             int n, int dh, int C, int P0, cudaStream_t s);
 
 // ---------------------------------------------------------------- elementwise / norm
 // h[t] = float(E[canvas[t]]) (or float(x_in[t]) when x_in != NULL);
@@ -159,6 +162,13 @@ struct AttnMergeArgs {
 struct AttnTcArgs {
   int B, Hq, Hkv, Tc, P, dh;
   int n_vis;
+  // Rows per (sequence, kv head) in the prompt K/V maps: P for a caller's cache,
+  // the capacity for the library's own.
+  int kv_stride;
+  // Causal attention (the encoder): new token i (position P + i) sees the cached
+  // and new positions <= P + i, and with window > 0 only those >= P + i - window + 1.
+  // n_vis then covers the widest row's cached range.  0: the decoder's joint softmax.
+  int causal, window;
   int n_chunks;          // key-block ranges per (canvas, kv head, query tile)
   float* part_o;         // [n_chunks][B*Hq*Tc][dh]
   float* part_ml;        // [n_chunks][B*Hq*Tc][2]

@@ -608,6 +608,35 @@ cudaError_t launch_commit(const float* conf, const int32_t* tok, int32_t* canvas
 
 namespace dg {
 
+// ---------------------------------------------------------------- KV append
+
+// Copy the new tokens' keys and values kc / vc [B][Hkv][n][dh] into the cache
+// [B][Hkv][C][dh] at positions P0 .. P0 + n - 1: one warp per (b, head, token)
+// row, 16 bytes per lane per step.
+__global__ void kv_append_kernel(const bf16* __restrict__ kc, const bf16* __restrict__ vc,
+                                 bf16* __restrict__ ck, bf16* __restrict__ cv, int rows, int n,
+                                 int dh, int C, int P0) {
+  griddep_wait();
+  griddep_launch();
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  const int bg = warp / n, i = warp % n;
+  const size_t src = (size_t)warp * dh;
+  const size_t dst = ((size_t)bg * C + P0 + i) * dh;
+  for (int e = lane * 8; e < dh; e += 32 * 8) {
+    *reinterpret_cast<uint4*>(ck + dst + e) = *reinterpret_cast<const uint4*>(kc + src + e);
+    *reinterpret_cast<uint4*>(cv + dst + e) = *reinterpret_cast<const uint4*>(vc + src + e);
+  }
+}
+
+cudaError_t launch_kv_append(const bf16* kc, const bf16* vc, bf16* ck, bf16* cv, int B, int Hkv,
+                             int n, int dh, int C, int P0, cudaStream_t s) {
+  if (dh % 8 != 0 || P0 + n > C) return cudaErrorInvalidValue;
+  const int rows = B * Hkv * n;
+  return launch_k(kv_append_kernel, dim3((rows + 7) / 8), dim3(256), 0, s, kc, vc, ck, cv, rows, n,
+                  dh, C, P0);
+}
+
 __global__ void set_int_kernel(int* p, int v) { *p = v; }
 
 cudaError_t launch_set_int(int* p, int v, cudaStream_t s) {

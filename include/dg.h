@@ -94,6 +94,10 @@ typedef struct dg_config {
                                 fp32 scale s per weight row, w = q * s, where
                                 s = max|w_bf16| / 448 and q = E4M3(w_bf16 / s) (fp32
                                 division, round to nearest even); activations stay bf16 */
+  int max_context;           /* capacity, in positions per sequence, of the library's own KV
+                                cache (dg_encode, dg_generate); 0 = none is allocated.  It
+                                takes max_batch * n_kv_heads * max_context * head_dim * 2
+                                bf16 values per layer */
 } dg_config;
 
 enum { DG_DTYPE_BF16 = 0, DG_DTYPE_FP8_E4M3 = 1 };
@@ -192,6 +196,52 @@ int dg_canvas_step_host(dg_ctx* ctx, int32_t* canvas_host, int batch, int steps_
  * slot is committed at the end.  canvas: dev int32 [batch][canvas_len], in
  * place.  Ends with a synchronisation and reports device errors. */
 int dg_denoise_block(dg_ctx* ctx, int32_t* canvas, int batch, int n_steps);
+
+/* Pages: "Hands-On with Diffusion Gemma", How Is This Different from Previous
+ * Models? (the causal part ingests the input once and builds the state the
+ * canvas reads; after 256 tokens the model returns to causal context building)
+ * and Detailed Specs (Encoder and Decoder: unidirectional causal attention,
+ * KV cache relayed to the decoder; weight sharing); "DiffusionGemma: The
+ * Diffusion Era Begins ...", DiffusionGemma's Technical Architecture (the
+ * autoregressive encoder creates the prompt's KV cache).
+ * The causal encoder: runs n tokens per sequence (tokens: host or dev int32
+ * [batch][n], read during the call) through every block with the decoder's
+ * weights and causal attention (position p sees positions <= p; a local layer
+ * only the last `window` of them), after the positions already encoded, and
+ * appends each layer's rotated keys and values to the library's own KV cache.
+ * Then every layer's prompt K/V is that cache (replacing dg_set_prompt_kv's),
+ * so a following dg_canvas_step / dg_denoise_block cross-attends to all encoded
+ * positions with canvas row i at position (length + i).  Needs max_context > 0;
+ * the batch must equal the encoded context's; length + n <= max_context.
+ * DG_ERR_BAD_STATE without weights or without an own cache.  Synchronous at
+ * the end (device errors reported). */
+int dg_encode(dg_ctx* ctx, const int32_t* tokens, int batch, int n);
+
+/* Pages: as dg_encode.  Empties the library's own KV cache (length 0); the
+ * next dg_encode starts at position 0 and may use another batch. */
+int dg_reset_context(dg_ctx* ctx);
+
+/* Pages: as dg_encode.  *n_out = positions per sequence in the own KV cache. */
+int dg_context_length(dg_ctx* ctx, int* n_out);
+
+/* Pages: as dg_encode.  Copies one layer's own cache, the positions encoded so
+ * far: k_out, v_out (host or dev) bf16 [batch][n_kv_heads][length][head_dim],
+ * keys rotated.  Synchronous.  DG_ERR_BAD_STATE when nothing is encoded. */
+int dg_context_kv(dg_ctx* ctx, int layer, void* k_out, void* v_out);
+
+/* Pages: "Hands-On with Diffusion Gemma", How Is This Different from Previous
+ * Models? (causal context building, then non-causal refinement of a 256-token
+ * canvas, repeated until the text is complete); "DiffusionGemma: Google's
+ * Experimental Diffusion LLM", How Text Diffusion Actually Works (a fixed
+ * number of passes per block).
+ * Block-autoregressive generation: empties the own cache, encodes the prompt
+ * (host or dev int32 [batch][n_prompt]), then n_blocks times: an all-mask
+ * canvas gets n_steps fixed passes (dg_denoise_block) against the cache, is
+ * written to out[:, blk * canvas_len ...] (host or dev int32
+ * [batch][n_blocks * canvas_len]) and is encoded onto the cache.  Needs
+ * n_prompt + n_blocks * canvas_len <= max_context.  Synchronous. */
+int dg_generate(dg_ctx* ctx, const int32_t* prompt, int batch, int n_prompt, int n_blocks,
+                int n_steps, int32_t* out);
 
 /* Pages: "DiffusionGemma: The Diffusion Era Begins with 4x Faster Text
  * Generation", Recommended Inference Settings (an entropy-bound sampler, at most

@@ -20,7 +20,8 @@ def rel_l2(a, b) -> float:
 class Ctx:
     """A libdg context with seeded weights and the prompt K/V of every layer."""
 
-    def __init__(self, cfg: dict, max_batch=None, max_prompt=None, with_prompt=True):
+    def __init__(self, cfg: dict, max_batch=None, max_prompt=None, with_prompt=True,
+                 max_context=0):
         import canvas_denoising_step_b200 as dg
         self.dg, self.cfg = dg, cfg
         self.B, self.Tc, self.P = cfg["batch"], cfg["canvas_len"], cfg["prompt_len"]
@@ -30,7 +31,8 @@ class Ctx:
         self.prev_stream = torch.cuda.current_stream()
         torch.cuda.set_stream(self.torch_stream)
         self.stream = self.torch_stream.cuda_stream
-        self.ctx = dg.dg_create(dg.config_from_dict(cfg, max_batch, max_prompt), self.stream)
+        self.ctx = dg.dg_create(dg.config_from_dict(cfg, max_batch, max_prompt,
+                                                    max_context=max_context), self.stream)
         dg.dg_init_weights(self.ctx, cfg["seed"])
         self.kv_host, self.kv_dev = [], []
         if with_prompt:

@@ -67,6 +67,10 @@ def test_invalid_configs_rejected_before_device_use(dg):
         assert rc == dg.DG_ERR_INVALID_ARG, b
         assert out.value is None
         assert dg.dg_last_error(None) != ""
+    cfg = dg.config_from_dict(base, max_context=-1)
+    out = ctypes.c_void_p()
+    assert dg.raw_call("dg_create", ctypes.byref(cfg), None, ctypes.byref(out)) == \
+        dg.DG_ERR_INVALID_ARG
 
 
 def test_configs_whose_router_grouping_cannot_fit_are_rejected(dg):
@@ -107,7 +111,11 @@ def test_null_arguments_and_no_device(dg):
                        ("dg_layer_forward", (None, 0, None, None, 1)),
                        ("dg_set_prompt_kv", (None, 0, None, None, 1, 1)),
                        ("dg_router_topk", (None, None, 1, None, None, None, None)),
-                       ("dg_commit", (None, None, None, 1, 1, None, None))]:
+                       ("dg_commit", (None, None, None, 1, 1, None, None)),
+                       ("dg_encode", (None, None, 1, 1)), ("dg_reset_context", (None,)),
+                       ("dg_context_length", (None, None)),
+                       ("dg_context_kv", (None, 0, None, None)),
+                       ("dg_generate", (None, None, 1, 1, 1, 1, None))]:
         assert dg.raw_call(name, *args) == dg.DG_ERR_INVALID_ARG, name
     dg.dg_destroy(None)
     assert dg.dg_device_bytes(None) == 0
