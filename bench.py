@@ -798,6 +798,16 @@ def run_encode_case(args, cfg):
         chunk = mb * Tc // B
         n_chunks = -(-P // chunk)
         active = (float(act.sum().item()) - act0) / (args.steps * n_chunks * L)
+        # per-kernel times: one more round with every launch bracketed by events
+        dg.dg_profile_enable(ctx, 1)
+        run(args.steps)
+        kern, i = {}, 0
+        while (name := dg.dg_kernel_name(i)) is not None:
+            tot, cnt = dg.dg_profile_read(ctx, name)
+            if cnt:
+                kern[name] = tot / args.steps
+            i += 1
+        dg.dg_profile_enable(ctx, 0)
         dg.dg_destroy(ctx)
     peaks = load_peaks()
     nbytes, _ = encoder_bytes(cfg, active, chunk)
@@ -823,6 +833,7 @@ def run_encode_case(args, cfg):
                             "bound": "tensor" if flops_ms > bytes_ms else "hbm",
                             "peak": tflops if flops_ms > bytes_ms else hbm,
                             "peak_source": peaks[2]},
+        "kernels_ms_per_step": dict(sorted(kern.items(), key=lambda kv: -kv[1])),
         "clocks": clk}), flush=True)
 
 
