@@ -128,6 +128,10 @@ struct dg_ctx {
   // sets DG_CTA_PAIR=1: co-resident two-CTA clusters, 0 when off.  Measured
   // slower than the one-SM engine on every workload here, so off by default.
   int pair_clusters = 0;
+  // the router with its logits GEMM in one cluster kernel, when the environment sets
+  // DG_FUSED_ROUTER=1: parity-green, but the pass measured slower than with the logits
+  // GEMM and the router kernel apart (6.72 vs 6.56 ms on the stack), so off by default
+  bool fused_router = false;
   // Encoded context in the library's own KV cache (dg_encode / dg_generate):
   // positions held, and the batch they belong to (0: none yet).
   int ctx_len = 0, ctx_batch = 0;
@@ -434,8 +438,12 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next, int Tc, bool causal)
   DG_LAUNCH(c, K_POST_ATTN, launch_post_attn(c->part, splits, T, d, L.ln_post, L.ln_ff, cf.rms_eps, c->h,
                                 c->xperm, c->stream));
 
-  // router
-  if ((rc = run_dense(c, K_GEMM_ROUTER, L.m_r, c->m_x2_b, nullptr, E, T, d, &splits)) != DG_OK) return rc;
+  // router: logits, top-k and grouping in one cluster kernel (E <= 128), or the
+  // logits GEMM then the router kernel
+  const bool fused_router = c->fused_router && E <= 128;
+  if (!fused_router &&
+      (rc = run_dense(c, K_GEMM_ROUTER, L.m_r, c->m_x2_b, nullptr, E, T, d, &splits)) != DG_OK)
+    return rc;
   {
     RouterArgs ra;
     memset(&ra, 0, sizeof(ra));
@@ -448,7 +456,16 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next, int Tc, bool causal)
     ra.chunk_ready = c->chunk_ready; ra.n_chunk_ready = c->n_chunk_ready;
     ra.chunk_order = c->chunk_order; ra.tile_counters = c->tile_counters; ra.n_tile_counters = 2;
     ra.perm = c->perm; ra.inv = c->inv; ra.active_out = c->expert_active + l; ra.err = c->err_dev;
-    DG_LAUNCH(c, K_ROUTER, launch_router(ra, c->stream));
+    if (fused_router) {
+      RouterFusedArgs rf;
+      memset(&rf, 0, sizeof(rf));
+      rf.r = ra;
+      rf.n_kb = d / 64;
+      rf.n_tile = c->dense_box;
+      DG_LAUNCH(c, K_ROUTER, launch_router_fused(L.m_r, c->m_x2_b, rf, c->stream));
+    } else {
+      DG_LAUNCH(c, K_ROUTER, launch_router(ra, c->stream));
+    }
   }
   DG_LAUNCH(c, K_GATHER, launch_moe_gather(c->xperm, c->perm, T, k, d, c->stream));
 
@@ -727,6 +744,8 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
   {
     const char* e = std::getenv("DG_CTA_PAIR");
     c->pair_clusters = (e && e[0] && e[0] != '0') ? gemm_pair_max_clusters() : 0;
+    const char* fr = std::getenv("DG_FUSED_ROUTER");
+    c->fused_router = fr && fr[0] && fr[0] != '0';
   }
   const dg_config& cf = c->cfg;
   const int d = cf.d_model, F = cf.d_ff, dh = cf.head_dim, E = cf.n_experts, k = cf.top_k;

@@ -225,6 +225,20 @@ struct RouterArgs {
 size_t router_smem_bytes(int T, int E);
 int router_max_smem_bytes();   // launch_router refuses larger shared-memory plans
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t s);
+// The router with its logits GEMM (E <= 128): logits = X W^T on the tensor cores,
+// split over the hidden dimension across a cluster of min(8, n_kb) CTAs per tile of
+// n_tile token rows and summed in rank order through distributed shared memory;
+// then top-k and the grouping as launch_router.  mapW: the router weights
+// [>=128][d] bf16 (128-row boxes), mapX: the normed rows [T..][d] (n_tile-row boxes).
+// logits_in / splits of r are not used.
+struct RouterFusedArgs {
+  RouterArgs r;
+  int n_kb;         // d / 64
+  int n_tile;       // token rows per cluster (the B box height), a multiple of 16, <= 256
+  int ring_bytes;   // set by the launcher
+};
+cudaError_t launch_router_fused(const CUtensorMap& mapW, const CUtensorMap& mapX,
+                                RouterFusedArgs f, cudaStream_t s);
 // xperm[T + p] = xperm[perm[p] / k] for p < k*T (rows [0, T) hold the normed input).
 cudaError_t launch_moe_gather(bf16* xperm, const int32_t* perm, int T, int k, int d,
                               cudaStream_t s);
