@@ -31,6 +31,9 @@
 // Every wait is bounded (kWaitLimitNs); both CTAs meet at a cluster barrier
 // before either frees TMEM or exits, so no CTA leaves while its peer can
 // still reach its shared memory.
+#include <map>
+#include <mutex>
+
 #include "gemm_shared.cuh"
 
 namespace dg {
@@ -479,8 +482,17 @@ size_t gemm_pair_smem_bytes(const GemmArgs& a) {
 }
 
 int gemm_pair_max_clusters() {
-  static int cached = -1;
-  if (cached < 0) {
+  // per device, as the occupancy it answers
+  static std::mutex mu;
+  static std::map<int, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(dev);
+  if (it == cache.end()) {
     int n = 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2);
@@ -499,9 +511,9 @@ int gemm_pair_max_clusters() {
       cudaGetLastError();
       n = 0;
     }
-    cached = n;
+    it = cache.emplace(dev, n).first;
   }
-  return cached;
+  return it->second;
 }
 
 cudaError_t gemm_pair_launch(const CUtensorMap& mapA, const CUtensorMap& mapB_half,
