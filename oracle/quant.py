@@ -3,8 +3,8 @@ path imports this module).
 
 "DiffusionGemma: The Diffusion Era Begins with 4x Faster Text Generation",
 Comparison with Other Models and Approaches, names low-precision (NVFP4) kernels
-for the model on Hopper and Blackwell; SURVEY's next row asks for NVFP4 or FP8
-expert weights.  The reading taken here: FP8 E4M3 expert weights with one fp32
+for the model on Hopper and Blackwell, which cut the bytes of the expert weights
+that dominate a pass.  The reading taken here: FP8 E4M3 expert weights with one fp32
 scale per output row (per channel), activations kept in bf16.  For a weight row
 w (the bf16 values of the seeded generator, read as float32):
 
