@@ -49,3 +49,36 @@ def test_clock_sample_stamps_parse():
     t2 = bench.ClockSampler._stamp("2026/12/02 17:10:02.000")
     assert t2 - t == pytest.approx(0.75)
     assert bench.ClockSampler._stamp("not a time") is None
+
+
+def test_encoder_flops_count_each_position_once_per_visible_key():
+    """Brute force on a small shape: per layer, every position's projections and experts,
+    plus causal attention over the positions it sees (window on local layers)."""
+    import synth
+    cfg = synth.config("tiny", prompt_len=37, window=5, global_every=2)
+    d, F, E, k = cfg["d_model"], cfg["d_ff"], cfg["n_experts"], cfg["top_k"]
+    dh, Hq, Hkv, P, W = cfg["head_dim"], cfg["n_q_heads"], cfg["n_kv_heads"], 37, 5
+    per_token = 2 * ((Hq + 2 * Hkv) * dh * d + d * Hq * dh + E * d) + 2 * (k + 1) * 3 * F * d
+    want = 0
+    for l in range(cfg["n_layers"]):
+        glob = (l + 1) % cfg["global_every"] == 0
+        for p in range(P):
+            seen = p + 1 if glob else min(p + 1, W)
+            want += per_token + 4 * Hq * dh * seen
+    assert bench.encoder_flops(cfg) == want * cfg["batch"]
+
+
+def test_encoder_bytes_read_each_chunks_weights_once_and_the_visible_cache():
+    """Two chunks of 16 over a 20-token prompt: weights twice per layer, the second chunk
+    reads the first chunk's cache (all of it on the global layer, window - 1 on the local)."""
+    import synth
+    cfg = synth.config("tiny", prompt_len=20, window=5, global_every=2)
+    d, F, E = cfg["d_model"], cfg["d_ff"], cfg["n_experts"]
+    dh, Hq, Hkv, L, B = cfg["head_dim"], cfg["n_q_heads"], cfg["n_kv_heads"], 2, cfg["batch"]
+    dense = 2 * ((Hq + 2 * Hkv) * dh * d + d * Hq * dh + E * d)
+    egb = 3 * F * d * 2
+    kv_row = 2 * B * Hkv * dh * 2            # one position's K and V, every kv head
+    kv = (0 + 16) * kv_row + (4 + 4) * kv_row + (0 + 16) * kv_row + (16 + 4) * kv_row
+    want = 2 * L * dense + 2 * L * (3 + 1) * egb + kv + B * 20 * d * 2
+    got, n_chunks = bench.encoder_bytes(cfg, 3, chunk=16)
+    assert n_chunks == 2 and got == want
