@@ -21,9 +21,20 @@
 //                    stale m is kept (P <= 256 stays exact enough in bf16);
 //                    write P_j as bf16 into shared memory in the K-major
 //                    128-byte-swizzle layout the MMA reads.
-// The CTA writes the un-normalised partial (O, m, l) of its key range; the
-// log-sum-exp merge kernel combines the ranges.
+// The CTA's result is the un-normalised partial (O, m, l) of its key range.
+// With the in-cluster merge (the key ranges of one query tile launched as one
+// thread-block cluster of at most 8 CTAs) every CTA stages its partial in its own
+// shared memory, and after a cluster barrier CTA c combines rows
+// [128c/C, 128(c+1)/C) of all C partials by log-sum-exp, reading its peers'
+// shared memory (distributed shared memory), and writes the bf16 output the
+// output projection reads; a second cluster barrier keeps every CTA resident
+// until its peers have read it.  Otherwise the partials go to global memory and
+// the merge kernel (attn_merge.cu) combines them, with the same arithmetic in the
+// same order, so the two routes give the same bits.
 #include <climits>
+#include <map>
+#include <mutex>
+#include <tuple>
 
 #include "dg_kernels.h"
 
@@ -36,6 +47,41 @@ constexpr int kBN = 64;          // keys per block
 constexpr int kRows = 128;       // query rows per CTA
 constexpr int kStages = 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kMaxClusterChunks = 8;       // key ranges merged inside one cluster
+constexpr int kWStride = kMaxClusterChunks + 1;   // a merged row's weights, then 1 / L
+
+__device__ __forceinline__ uint32_t attn_cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// the address of the same shared-memory location in the cluster's CTA `rank`
+__device__ __forceinline__ uint32_t attn_mapa(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ float4 attn_ld_cluster_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ float2 attn_ld_cluster_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
+  return v;
+}
+
+// every thread of every CTA of the cluster; the writes before it are seen after it
+__device__ __forceinline__ void attn_cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
 
 template <int DH>
 struct AttnSmem {
@@ -48,9 +94,114 @@ struct AttnSmem {
   static constexpr int kPOff = kVOff + kStages * kKV;   // [2] P tiles
   static constexpr int kBarOff = kPOff + 2 * kP;
   static constexpr int kBytes = kBarOff + 256;
+  // in-cluster merge, over the operand buffers once every MMA has finished:
+  // the partial O [128 rows][DH] fp32 (16-byte chunk k of row r at k ^ (r % 8)),
+  // the rows' (m, l), and per merged row the chunks' weights and 1 / L
+  static constexpr int kStageOff = 0;
+  static constexpr int kMlOff = kStageOff + kRows * DH * 4;
+  static constexpr int kWOff = kMlOff + kRows * 8;
+  static_assert(kWOff + kRows * kWStride * 4 <= kBarOff, "merge staging overlaps the barriers");
 };
 
 }  // namespace
+
+// The in-cluster log-sum-exp merge (every thread of the CTA calls it).  The CTA of
+// rank c holds key range c's partial (the cluster spans the grid's y dimension,
+// so the rank is blockIdx.y).  For each of its rows [128c/C, 128(c+1)/C):
+// M = max_c m_c, w_c = 2^(m_c - M) (0 for a range that saw no key),
+// L = sum_c w_c l_c and o = (sum_c w_c O_c) / L, the sums in the order the merge
+// kernel takes them (L as a 32-lane butterfly, O in range order), fp32 with
+// every rounding explicit.
+template <int DH>
+__device__ __forceinline__ void attn_cluster_merge(const AttnTcArgs& a, uint8_t* smem, uint32_t sbase,
+                                                   int qt, int b, int g) {
+  using L = AttnSmem<DH>;
+  constexpr int KC = DH / 4;          // 16-byte chunks per row
+  constexpr int kU = 4;               // items whose loads are in flight together
+  const int C = a.n_chunks;
+  const int group = a.Hq / a.Hkv;
+  const int q_rows = group * a.Tc;
+  const int me = (int)attn_cluster_rank();
+  const int row0 = me * kRows / C, row1 = (me + 1) * kRows / C;
+  const int nrows = row1 - row0;
+  float* sw = reinterpret_cast<float*>(smem + L::kWOff);
+  attn_cluster_sync();                // every CTA of the cluster has staged its partial
+  for (int t = threadIdx.x; t < nrows; t += blockDim.x) {
+    const int r = row0 + t;
+    float mc[kMaxClusterChunks], lc[kMaxClusterChunks];
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kMaxClusterChunks; ++c) {
+      mc[c] = -INFINITY;
+      lc[c] = 0.f;
+      if (c < C) {
+        const float2 ml = attn_ld_cluster_f2(attn_mapa(sbase + L::kMlOff + (uint32_t)r * 8u, (uint32_t)c));
+        mc[c] = ml.x;
+        lc[c] = ml.y;
+        M = fmaxf(M, ml.x);
+      }
+    }
+    float wl[kMaxClusterChunks];
+#pragma unroll
+    for (int c = 0; c < kMaxClusterChunks; ++c) {
+      const float w = (mc[c] == -INFINITY) ? 0.f : exp2f(__fsub_rn(mc[c], M));
+      sw[t * kWStride + c] = w;
+      wl[c] = __fmul_rn(w, lc[c]);
+    }
+    // a 32-lane xor butterfly over the ranges' w l (zero past C) adds, in lane 0,
+    // ((v0 + v4) + (v2 + v6)) + ((v1 + v5) + (v3 + v7))
+    const float Ls = __fadd_rn(__fadd_rn(__fadd_rn(wl[0], wl[4]), __fadd_rn(wl[2], wl[6])),
+                               __fadd_rn(__fadd_rn(wl[1], wl[5]), __fadd_rn(wl[3], wl[7])));
+    sw[t * kWStride + kMaxClusterChunks] = __frcp_rn(Ls);
+  }
+  __syncthreads();
+  const int items = nrows * KC;
+  for (int i0 = threadIdx.x; i0 < items; i0 += kU * (int)blockDim.x) {
+    float4 acc[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < C; ++c) {
+      float4 o[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int it = i0 + u * (int)blockDim.x;
+        if (it < items) {
+          const int r = row0 + it / KC, k = it % KC;
+          o[u] = attn_ld_cluster_f4(attn_mapa(sbase + L::kStageOff + (uint32_t)r * (DH * 4) +
+                                                  (uint32_t)((k ^ (r & 7)) * 16),
+                                              (uint32_t)c));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int it = i0 + u * (int)blockDim.x;
+        if (it < items) {
+          const float w = sw[(it / KC) * kWStride + c];
+          acc[u].x = __fmaf_rn(w, o[u].x, acc[u].x);
+          acc[u].y = __fmaf_rn(w, o[u].y, acc[u].y);
+          acc[u].z = __fmaf_rn(w, o[u].z, acc[u].z);
+          acc[u].w = __fmaf_rn(w, o[u].w, acc[u].w);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int it = i0 + u * (int)blockDim.x;
+      if (it >= items) continue;
+      const int rr = it / KC, k = it % KC;
+      const int qr = qt * kRows + row0 + rr;
+      if (qr >= q_rows) continue;
+      const int h = g * group + qr / a.Tc, i = qr % a.Tc;
+      const float inv = sw[rr * kWStride + kMaxClusterChunks];
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(__fmul_rn(acc[u].x, inv), __fmul_rn(acc[u].y, inv));
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(__fmul_rn(acc[u].z, inv), __fmul_rn(acc[u].w, inv));
+      bf16* dst = a.out + ((size_t)b * a.Tc + i) * ((size_t)a.Hq * DH) + (size_t)h * DH + 4 * k;
+      *reinterpret_cast<uint2*>(dst) =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+    }
+  }
+  attn_cluster_sync();                // no CTA leaves while a peer still reads it
+}
 
 template <int DH>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -384,6 +535,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
     if (ok && n_local > 0)
       ok = mbar_wait(pv_done((n_local - 1) & 1), (uint32_t)(((n_local - 1) >> 1) & 1), abort_flag, a.err);
     tc_fence_after();
+    if (a.fused) {
+      // stage the partial for the cluster's merge: this thread's row r, 32 columns per
+      // TMEM load, 16-byte chunk k at k ^ (r % 8) (eight consecutive rows cover all banks)
+      const uint32_t srow = sbase + L::kStageOff + (uint32_t)r * (DH * 4);
+#pragma unroll 1
+      for (int c0 = 0; c0 < DH; c0 += 32) {
+        if (n_local > 0 && ok) {
+          tmem_ld32(lane_base + kOCol + c0, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        }
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4)
+          st_shared_v4(srow + (uint32_t)((((c0 >> 2) + c4) ^ (r & 7)) * 16), v[4 * c4], v[4 * c4 + 1],
+                       v[4 * c4 + 2], v[4 * c4 + 3]);
+      }
+      reinterpret_cast<float2*>(smem + L::kMlOff)[r] = make_float2((n_local > 0) ? m : -INFINITY, l);
+    } else {
     const int qr = qt * kRows + r;
     const int rows_total = a.B * a.Hq * a.Tc;
     const bool row_valid = qr < q_rows;
@@ -439,6 +610,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
       pml[0] = (n_local > 0) ? m : -INFINITY;
       pml[1] = l;
     }
+    }
   }
 
   tc_fence_before();
@@ -447,6 +619,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  // every thread of every CTA reaches this point on every path (no early exit), so
+  // the cluster barriers inside always complete
+  if (a.fused) attn_cluster_merge<DH>(a, smem, sbase, qt, b, g);
 }
 
 namespace {
@@ -458,11 +633,77 @@ cudaError_t launch_attn_tc_t(const AttnTcMaps& m, const AttnTcArgs& a, cudaStrea
   if (e != cudaSuccess) return e;
   const int group = a.Hq / a.Hkv;
   dim3 grid((group * a.Tc + kRows - 1) / kRows, a.n_chunks, a.B * a.Hkv);
-  return launch_k(attn_tc_kernel<DH>, grid, dim3(kThreads), smem, s, m.q, m.kc, m.vc, m.kp, m.vp,
-                  m.po, a);
+  if (!a.fused)
+    return launch_k(attn_tc_kernel<DH>, grid, dim3(kThreads), smem, s, m.q, m.kc, m.vc, m.kp, m.vp,
+                    m.po, a);
+  if (a.n_chunks < 1 || a.n_chunks > kMaxClusterChunks || a.out == nullptr) return cudaErrorInvalidValue;
+  // the key ranges of one query tile form one cluster along y
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = (unsigned)a.n_chunks;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, attn_tc_kernel<DH>, m.q, m.kc, m.vc, m.kp, m.vp, m.po, a);
+}
+
+template <int DH>
+int attn_fused_clusters_t(int n_chunks) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, (unsigned)n_chunks, 1);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = AttnSmem<DH>::kBytes + 1024;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = (unsigned)n_chunks;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (ensure_smem_limit(reinterpret_cast<const void*>(attn_tc_kernel<DH>),
+                        (int)(AttnSmem<DH>::kBytes + 1024)) != cudaSuccess ||
+      cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel<DH>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  return n;
 }
 
 }  // namespace
+
+bool attn_tc_fused_ok(int dh, int n_chunks) {
+  if (n_chunks < 1 || n_chunks > kMaxClusterChunks) return false;
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int>, int> cache;   // (device, dh, chunks) -> clusters
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  auto key = std::make_tuple(dev, dh, n_chunks);
+  auto it = cache.find(key);
+  if (it == cache.end()) {
+    int n = 0;
+    switch (dh) {
+      case 64: n = attn_fused_clusters_t<64>(n_chunks); break;
+      case 128: n = attn_fused_clusters_t<128>(n_chunks); break;
+      case 256: n = attn_fused_clusters_t<256>(n_chunks); break;
+      default: n = 0;
+    }
+    it = cache.emplace(key, n).first;
+  }
+  return it->second > 0;
+}
 
 int attn_tc_blocks(int n_vis, int Tc) { return (n_vis + kBN - 1) / kBN + (Tc + kBN - 1) / kBN; }
 int attn_tc_qtiles(int Hq, int Hkv, int Tc) { return (Hq / Hkv * Tc + kRows - 1) / kRows; }

@@ -2,7 +2,9 @@
 // chunks' (O, m, l) (m in log2 units) combine by log-sum-exp into
 // o = sum_c 2^{m_c - M} O_c / sum_c 2^{m_c - M} l_c, written as bf16 into the
 // [T][Hq * dh] layout that the output projection reads.  One warp per row,
-// lane c holding chunk c's (m, l) (at most 32 chunks).
+// lane c holding chunk c's (m, l) (at most 32 chunks).  Every rounding is
+// explicit (no contraction), so the attention kernel's in-cluster merge, which
+// takes the same steps in the same order, gives the same bits.
 #include "dg_kernels.h"
 
 namespace dg {
@@ -44,8 +46,8 @@ __global__ void attn_merge_kernel(const AttnMergeArgs a, bf16* out) {
                         : make_float2(0.f, 0.f);
     if (c0 == 0) {
       M = warp_max(mc);
-      wl = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
-      L = warp_sum(wl * lc);
+      wl = (mc == -INFINITY) ? 0.f : exp2f(__fsub_rn(mc, M));
+      L = warp_sum(__fmul_rn(wl, lc));
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
@@ -53,8 +55,8 @@ __global__ void attn_merge_kernel(const AttnMergeArgs a, bf16* out) {
       if (c0 + u < nc)
 #pragma unroll
         for (int j = 0; j < NJ; ++j) {
-          acc[j].x += wgt * buf[u][j].x;
-          acc[j].y += wgt * buf[u][j].y;
+          acc[j].x = __fmaf_rn(wgt, buf[u][j].x, acc[j].x);
+          acc[j].y = __fmaf_rn(wgt, buf[u][j].y, acc[j].y);
         }
     }
   }
@@ -62,11 +64,11 @@ __global__ void attn_merge_kernel(const AttnMergeArgs a, bf16* out) {
   const int bh = R / a.Tc;
   const int h = bh % a.Hq, b = bh / a.Hq;
   bf16* dst = out + ((size_t)b * a.Tc + i) * ((size_t)a.Hq * DH) + (size_t)h * DH;
-  const float inv = 1.0f / L;
+  const float inv = __frcp_rn(L);
 #pragma unroll
   for (int j = 0; j < NJ; ++j)
     *reinterpret_cast<__nv_bfloat162*>(dst + 2 * lane + 64 * j) =
-        __floats2bfloat162_rn(acc[j].x * inv, acc[j].y * inv);
+        __floats2bfloat162_rn(__fmul_rn(acc[j].x, inv), __fmul_rn(acc[j].y, inv));
 }
 
 }  // namespace

@@ -132,6 +132,13 @@ struct dg_ctx {
   // DG_FUSED_ROUTER=1: parity-green, but the pass measured slower than with the logits
   // GEMM and the router kernel apart (6.72 vs 6.56 ms on the stack), so off by default
   bool fused_router = false;
+  // The attention's key ranges merged inside a thread-block cluster (no partials
+  // through global memory, no merge kernel), when the environment sets
+  // DG_ATTN_CLUSTER_MERGE=1.  Both routes give the same bits; on the stack the
+  // cluster route measured slower (6.66 against 6.57 ms per pass: its merge phase
+  // adds ~7 µs to each attention launch, while the merge kernel it replaces costs
+  // less than that inside the graph), so the merge kernel is the default.
+  bool attn_cluster_merge = false;
   // Encoded context in the library's own KV cache (dg_encode / dg_generate):
   // positions held, and the batch they belong to (0: none yet).
   int ctx_len = 0, ctx_batch = 0;
@@ -420,15 +427,19 @@ int run_layer(dg_ctx* c, int l, int B, const float* w_next, int Tc, bool causal)
   ta.part_o = c->attn_po; ta.part_ml = c->attn_ml;
   ta.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)dh));
   ta.err = c->err_dev;
+  ta.out = c->attn_o;
+  ta.fused = (c->attn_cluster_merge && attn_tc_fused_ok(dh, ta.n_chunks)) ? 1 : 0;
   AttnTcMaps tm;
   tm.q = c->m_q; tm.kc = c->m_kc; tm.vc = c->m_vc; tm.kp = L.m_kp; tm.vp = L.m_vp;
   tm.po = c->m_attn_po;
   DG_LAUNCH(c, K_ATTN, launch_attention_tc(tm, ta, c->stream));
-  AttnMergeArgs at;
-  at.B = B; at.Hq = Hq; at.Tc = Tc; at.dh = dh;
-  at.n_chunks = ta.n_chunks;
-  at.part_o = c->attn_po; at.part_ml = c->attn_ml;
-  DG_LAUNCH(c, K_ATTN_MERGE, launch_attn_merge(at, c->attn_o, c->stream));
+  if (!ta.fused) {
+    AttnMergeArgs at;
+    at.B = B; at.Hq = Hq; at.Tc = Tc; at.dh = dh;
+    at.n_chunks = ta.n_chunks;
+    at.part_o = c->attn_po; at.part_ml = c->attn_ml;
+    DG_LAUNCH(c, K_ATTN_MERGE, launch_attn_merge(at, c->attn_o, c->stream));
+  }
   if (causal)
     DG_LAUNCH(c, K_KV_APPEND, launch_kv_append(c->kc, c->vc, L.own_k, L.own_v, B, Hkv, Tc, dh,
                                                cf.max_context, P, c->stream));
@@ -746,6 +757,11 @@ int dg_create(const dg_config* cfg, void* cuda_stream, dg_ctx** out) {
     c->pair_clusters = (e && e[0] && e[0] != '0') ? gemm_pair_max_clusters() : 0;
     const char* fr = std::getenv("DG_FUSED_ROUTER");
     c->fused_router = fr && fr[0] && fr[0] != '0';
+    const char* cm = std::getenv("DG_ATTN_CLUSTER_MERGE");
+    c->attn_cluster_merge = cm && cm[0] && cm[0] != '0';
+    // whether each cluster size fits is asked once here, outside any graph capture
+    if (c->attn_cluster_merge)
+      for (int n = 1; n <= 8; ++n) attn_tc_fused_ok(c->cfg.head_dim, n);
   }
   const dg_config& cf = c->cfg;
   const int d = cf.d_model, F = cf.d_ff, dh = cf.head_dim, E = cf.n_experts, k = cf.top_k;

@@ -174,6 +174,10 @@ struct AttnTcArgs {
   float* part_ml;        // [n_chunks][B*Hq*Tc][2]
   float scale_log2;
   int* err;
+  // 1: the n_chunks CTAs of a query tile run as one cluster and merge in shared
+  // memory into `out` (n_chunks <= 8; part_o / part_ml unused); 0: partials
+  int fused;
+  bf16* out;             // [T][Hq*dh] bf16 (t = b*Tc + i), as the merge kernel writes
 };
 struct AttnTcMaps {
   CUtensorMap q;         // [B*Hq*Tc][dh], box 64 x 128 rows
@@ -184,6 +188,9 @@ struct AttnTcMaps {
 int attn_tc_blocks(int n_vis, int Tc);
 int attn_tc_qtiles(int Hq, int Hkv, int Tc);
 cudaError_t launch_attention_tc(const AttnTcMaps& m, const AttnTcArgs& a, cudaStream_t s);
+// Whether the cluster-merged form can run with this head width and range count on
+// the current device (at most 8 ranges, and the cluster fits the GPU).
+bool attn_tc_fused_ok(int dh, int n_chunks);
 // Merge partials -> o [T][Hq*dh] bf16 (t = b*Tc + i)
 cudaError_t launch_attn_merge(const AttnMergeArgs& a, bf16* o, cudaStream_t s);
 
